@@ -1,0 +1,321 @@
+#!/usr/bin/env python
+"""Benchmark: batch-1 greedy decode (tg128) after a 520-token prompt (pp520)
+on the 0.8B-shaped hybrid DeltaNet/attention model, synthetic bf16 weights.
+
+One step = mk_reset + mk_prefill(520 prompt tokens) + mk_generate(128 greedy
+tokens, device-resident loop).  `value` is decode tokens/s over all ranks
+(replicas: one independent engine per GPU, no collective on the data path);
+prefill tokens/s, the decode kernel's HBM roofline fraction, the
+end-to-end number through host buffers and the CPU oracle baseline ride on
+the same JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PROMPT = 520
+GEN = 128
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=3)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def decode_bytes(cfg, ctx):
+    """Algorithmic HBM bytes of one decode launch at context `ctx` (the new
+    token is position ctx): every weight once (tied embedding read as the LM
+    head), DeltaNet state read+write, conv history read+write, KV read of
+    ctx positions + write of one, logits written."""
+    import numpy as np
+    from attention_decode_megakernel_b200 import synth
+    n = 0
+    for is_attn in cfg.layer_is_attn:
+        for _, shape, kind in synth.layer_tensor_shapes(cfg, is_attn):
+            n += int(np.prod(shape)) * (4 if kind == "f" else 2)
+    n += cfg.vocab * cfg.hidden * 2 + cfg.hidden * 2
+    n += 2 * cfg.n_dn * cfg.dn_heads * cfg.dn_dv * cfg.dn_dk * 4
+    n += 2 * cfg.n_dn * cfg.conv_channels * (cfg.conv_k - 1) * 4
+    kv_pos = cfg.n_attn * 2 * cfg.kv_heads * cfg.head_dim * 2
+    n += kv_pos * (ctx + 1)
+    n += cfg.vocab * 4
+    return n
+
+
+class Clocks:
+    """nvidia-smi samples during the timed region (read-only)."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.f.name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def oracle_decode_rate(cfg, w, budget_s=12.0, max_steps=64):
+    """The fp64 oracle's decode tokens/s on this host at context 520 (state
+    installed from the seeded synthetic generator), timed for ~budget_s."""
+    import oracle
+    from attention_decode_megakernel_b200 import synth
+    m = oracle.OracleModel(cfg, w)
+    m.set_state(synth.make_engine_state(cfg, ctx=PROMPT))
+    tok, n, t0 = 1, 0, time.perf_counter()
+    while n < max_steps:
+        logits, _ = m.step(tok)
+        tok = int(logits.argmax())
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return n / dt, n, dt, cores
+
+
+def run_reference(args, rank):
+    """Reference arm: the CPU oracle as it stands, on the host cores."""
+    if rank != 0:
+        return
+    from attention_decode_megakernel_b200 import synth
+    cfg = synth.hybrid_08b_config(max_ctx=PROMPT + GEN + 8)
+    w = synth.make_weights(cfg)
+    import oracle
+    m = oracle.OracleModel(cfg, w)
+    st = synth.make_engine_state(cfg, ctx=PROMPT)
+    per_step = 4
+    times = []
+    for i in range(args.warmup + args.steps):
+        m.set_state(st)
+        tok = 1
+        t0 = time.perf_counter()
+        for _ in range(per_step):
+            logits, _ = m.step(tok)
+            tok = int(logits.argmax())
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = per_step * args.steps / total
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = ("%d greedy decode steps per bench step of the 0.8B-shaped model at "
+              "context 520 (seeded synthetic state), fp64 oracle" % per_step)
+    line = {
+        "impl": "reference", "metric": "batch-1 decode tok/s (tg128)", "value": value,
+        "unit": "tok/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "hybrid-0.8B-24L-h1024 pp520+tg128 (decode at ctx 520)",
+                   "prompt": PROMPT, "gen": GEN},
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import numpy as np
+    import torch
+
+    import attention_decode_megakernel_b200 as mk
+    from attention_decode_megakernel_b200 import build, synth
+
+    build.build()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    cfg = synth.hybrid_08b_config(max_ctx=PROMPT + GEN + 8)
+    w = synth.make_weights(cfg)
+    eng = mk.Engine(cfg, w)
+    prompt = synth.make_tokens(cfg.vocab, PROMPT)
+    toks = torch.zeros(GEN, dtype=torch.int32, device="cuda")
+    stream = eng.stream
+
+    def one_step(evs=None):
+        eng.reset()
+        if evs:
+            evs[0].record(stream)
+        eng.prefill(prompt)
+        if evs:
+            evs[1].record(stream)
+        eng.generate(-1, GEN, toks)
+        if evs:
+            evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    eng.sync()
+
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = Clocks(local)
+    clk.start()
+    launches0 = eng.launch_count()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        one_step(evs[k])
+    torch.cuda.synchronize()
+    eng.sync()
+    launches = eng.launch_count() - launches0
+    clocks = clk.stop()
+    if dist:
+        dist.barrier()
+    prefill_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    decode_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    if dist:
+        t = torch.tensor([prefill_ms, decode_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        prefill_ms, decode_ms = float(t[0]), float(t[1])
+    out_tokens = toks.cpu().numpy().tolist()
+
+    # end to end through the public API with host buffers: the first token
+    # comes from the host, the 128 generated tokens are read back into pinned
+    # host memory, both inside the timed region
+    host_toks = torch.zeros(GEN, dtype=torch.int32).pin_memory()
+    e2e_times = []
+    first = int(out_tokens[0])
+    for _ in range(args.steps):
+        eng.reset()
+        eng.prefill(prompt)
+        eng.sync()
+        t0 = time.perf_counter()
+        eng.generate(first, GEN, toks)
+        host_toks.copy_(toks, non_blocking=True)
+        stream.synchronize()
+        e2e_times.append(time.perf_counter() - t0)
+    e2e_s = sum(e2e_times)
+    if dist:
+        t = torch.tensor([e2e_s], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t[0])
+
+    hbm, _, peak_kind = peaks()
+    per_launch_s = decode_ms / 1000.0 / (GEN * args.steps)
+    bytes_avg = sum(decode_bytes(cfg, PROMPT + i) for i in range(GEN)) / GEN
+    achieved = bytes_avg / per_launch_s / 1e9
+    value = world * GEN * args.steps / (decode_ms / 1000.0)
+    prefill_tps = world * PROMPT * args.steps / (prefill_ms / 1000.0)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, n, dt, cores = oracle_decode_rate(cfg, w)
+        cpu = {"value": rate, "unit": "tok/s", "cores": cores, "kind": "oracle",
+               "sample": "%d greedy decode steps of the 0.8B-shaped model at context 520 "
+                         "(seeded synthetic state) in %.1f s, fp64 oracle" % (n, dt)}
+
+    line = {
+        "metric": "batch-1 decode tok/s (tg128)", "value": value, "unit": "tok/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": (prefill_ms + decode_ms) / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 weights, fp32 math",
+        "data": "synthetic (seeded N(0,0.02) bf16 weights, uniform random prompt)",
+        "config": {"workload": "hybrid-0.8B-24L-h1024 pp520+tg128", "prompt": PROMPT,
+                   "gen": GEN, "batch": 1, "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (1.33 GB streamed per token vs 126 MB L2)"},
+        "prefill_tok_s": prefill_tps,
+        "decode_ms_per_token": per_launch_s * 1000.0,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None, "peak_kind": peak_kind,
+                     "kernel": "decode_kernel (one launch per token)",
+                     "bytes_per_launch": bytes_avg},
+        "e2e": {"value": world * GEN * args.steps / e2e_s, "unit": "tok/s",
+                "h2d_bytes_per_step": 4, "d2h_bytes_per_step": GEN * 4},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+        "greedy_tokens_head": out_tokens[:8],
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    eng.close()
+    if dist:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

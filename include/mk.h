@@ -1,0 +1,215 @@
+/*
+ * mk.h -- C ABI of the single-launch decode engine for hybrid
+ * Gated-DeltaNet + full-attention language models on NVIDIA B200 (sm_100a).
+ *
+ * The operation behind every entry point is one token's (or a few tokens')
+ * forward pass of the hybrid stack described in the launch post "OS
+ * Megakernel that match M5 Max Tok/w at 2x the Throughput on RTX 3090"
+ * (paragraph "Why nobody had done this yet?": DeltaNet layers with a
+ * learned recurrence interleaved with full-attention layers; the kernel
+ * bullet list: one dispatch for the whole forward pass, bf16 weights,
+ * fp32 accumulation, fused QKV + RoPE + causal softmax + output
+ * projection, cooperative grid sync between layers).  The recurrence is
+ * the gated delta rule of "Gated Delta Networks" (Yang, Kautz &
+ * Hatamizadeh, ICLR 2025).
+ *
+ * Conventions shared by all entry points
+ *  - Every pointer documented as "device" must point to memory of the CUDA
+ *    device that was current when mk_create ran; "host" pointers are read
+ *    before the call returns.
+ *  - Calls are asynchronous on the stream given to mk_create unless stated.
+ *  - Nothing throws across the ABI.  Every call returns an mk_status code;
+ *    MK_OK is 0.  A device-side failure (a grid barrier or pipeline wait
+ *    that ran out of time) is recorded in a device error word and reported
+ *    by mk_sync(), and by the next call that synchronises.  After any error
+ *    the engine accepts only mk_reset() and mk_destroy(); mk_reset() clears
+ *    the error, the recurrent state and the KV cache.
+ *  - Tensors are row-major.  bf16 values are IEEE bfloat16 bit patterns.
+ */
+#ifndef MK_H
+#define MK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MK_MAX_LAYERS 64
+
+typedef enum {
+  MK_OK = 0,
+  MK_ERR_ARG = 1,          /* bad argument, shape, alignment or NULL        */
+  MK_ERR_CTX_OVERFLOW = 2, /* the call would write past max_ctx             */
+  MK_ERR_STATE = 3,        /* call not valid in the engine's current state  */
+  MK_ERR_LAUNCH = 4,       /* cooperative launch impossible / failed        */
+  MK_ERR_TIMEOUT = 5,      /* a device-side wait gave up (error word set)   */
+  MK_ERR_CUDA = 6,         /* another CUDA runtime error                    */
+  MK_ERR_UNSUPPORTED = 7   /* shape outside what the kernels implement      */
+} mk_status;
+
+/* Model shape.  Layer l is full attention when layer_is_attn[l] != 0 and a
+ * Gated-DeltaNet layer otherwise.  Shapes the kernels implement:
+ * hidden % 256 == 0 and <= 2048; dn_dk == dn_dv in {64, 128};
+ * head_dim in {64, 128, 256}; conv_k == 4; q_heads % kv_heads == 0 and
+ * q_heads / kv_heads <= 8; mlp % 8 == 0; the embedding is tied to the
+ * LM head.  mk_create returns MK_ERR_UNSUPPORTED otherwise. */
+typedef struct {
+  int32_t n_layers;
+  uint8_t layer_is_attn[MK_MAX_LAYERS];
+  int32_t hidden, vocab, mlp;
+  int32_t dn_heads, dn_dk, dn_dv, conv_k;
+  int32_t q_heads, kv_heads, head_dim;
+  float rope_theta, rms_eps;
+  int32_t max_ctx;     /* KV-cache capacity in positions                    */
+  int32_t max_verify;  /* most tokens one mk_verify call may carry (<= 8)   */
+} mk_config;
+
+/* Device pointers of one layer's weights.  bf16 matrices are [out][in];
+ * every pointer must be 16-byte aligned.  Members of the other layer kind
+ * are ignored and may be NULL.
+ *   attn_norm [H], mlp_norm [H]            pre-mixer / pre-MLP RMSNorm gains
+ *   in_proj   [2*nh*dk + 2*nh*dv + 2*nh][H] DeltaNet rows q | k | v | z | b | a
+ *   conv_w    [2*nh*dk + nh*dv][conv_k]    causal conv taps of q | k | v
+ *   A_log, dt_bias [nh] (float32)          decay parameters
+ *   out_norm  [dv]                         gated-RMSNorm gain (shared by heads)
+ *   out_proj  [H][nh*dv]                   DeltaNet output projection
+ *   w_q [q_heads*hd][H], w_k, w_v [kv_heads*hd][H], w_o [H][q_heads*hd]
+ *   w_gate, w_up [mlp][H], w_down [H][mlp] SwiGLU MLP                      */
+typedef struct {
+  const void *attn_norm;
+  const void *in_proj, *conv_w;
+  const float *A_log, *dt_bias;
+  const void *out_norm, *out_proj;
+  const void *w_q, *w_k, *w_v, *w_o;
+  const void *mlp_norm;
+  const void *w_gate, *w_up, *w_down;
+} mk_layer_weights;
+
+/* embed [vocab][H] bf16 (also the LM head: tied), final_norm [H] bf16,
+ * layers: host array of n_layers entries. */
+typedef struct {
+  const void *embed;
+  const void *final_norm;
+  const mk_layer_weights *layers;
+} mk_weights;
+
+typedef struct mk_engine mk_engine;
+
+/* Bytes of device workspace mk_create needs for this config (recurrent
+ * state, verify checkpoints, KV cache, activations, barrier words).
+ * Returns 0 for an invalid config. */
+size_t mk_workspace_bytes(const mk_config *cfg);
+
+/* Create an engine on the current CUDA device.  `workspace` (device, at
+ * least mk_workspace_bytes(cfg) bytes, 256-byte aligned) and the weights
+ * stay owned by the caller and must outlive the engine; the engine only
+ * keeps pointers.  `cuda_stream` (a cudaStream_t, may be NULL for the
+ * legacy stream) is the stream every later call runs on.  Checks that one
+ * CTA of the decode kernel fits on every SM (cooperative co-residency) and
+ * returns MK_ERR_LAUNCH otherwise.  Zeroes the state (as mk_reset). */
+int mk_create(const mk_config *cfg, const mk_weights *w, void *workspace,
+              size_t ws_bytes, void *cuda_stream, mk_engine **out);
+
+/* Destroy the host handle (NULL is allowed).  Does not free caller memory. */
+void mk_destroy(mk_engine *e);
+
+/* Zero the DeltaNet and conv states, empty the KV cache, clear a device
+ * error and any pending verify.  Weights are untouched. */
+int mk_reset(mk_engine *e);
+
+/* Run n prompt tokens (host array, values in [0, vocab)) through the stack
+ * at positions pos .. pos+n-1 and leave the state and KV cache as n decode
+ * steps would.  If logits_out (device, float32 [vocab]) is not NULL it
+ * receives the logits of the last prompt position.  n == 0 is a no-op.
+ * Errors: MK_ERR_CTX_OVERFLOW when pos+n > max_ctx. */
+int mk_prefill(mk_engine *e, const int32_t *tokens_host, int n,
+               float *logits_out);
+
+/* One decode step: one cooperative launch of the persistent kernel for
+ * `token` at the current position.  logits_out (device, float32 [vocab])
+ * may be NULL.  The greedy argmax of the step is kept on the device (see
+ * mk_generate) and can be read with mk_last_argmax. */
+int mk_decode_step(mk_engine *e, int32_t token, float *logits_out);
+
+/* Greedy generation with no host round trip between tokens: n decode
+ * launches, the first fed `first_token` (or, when first_token == -1, the
+ * device-side argmax of the previous launch, e.g. the last prefill
+ * position), each later one fed the device-side argmax of the launch before
+ * it.  tokens_out (device, int32 [n]) receives
+ * the n argmax tokens; logits_out (device, float32 [n][vocab]) may be NULL. */
+int mk_generate(mk_engine *e, int32_t first_token, int n, int32_t *tokens_out,
+                float *logits_out);
+
+/* Verify n tokens at once (1 <= n <= max_verify): the stack runs over
+ * positions pos .. pos+n-1 exactly as n decode steps would, writing the logits of every position to logits_out (device, float32
+ * [n][vocab], not NULL) and a checkpoint of the recurrent state after each
+ * position.  The position does not advance until mk_accept. */
+int mk_verify(mk_engine *e, const int32_t *tokens_host, int n,
+              float *logits_out);
+
+/* Keep the first n_keep (1..n) positions of the last mk_verify: the state
+ * becomes the checkpoint after position n_keep-1 and the position advances
+ * by n_keep.  MK_ERR_STATE if no verify is pending. */
+int mk_accept(mk_engine *e, int n_keep);
+
+/* Current position (number of tokens consumed). */
+int mk_position(const mk_engine *e);
+
+/* Synchronise the stream and report a recorded device-side error. */
+int mk_sync(mk_engine *e);
+
+/* Host copy of the packed argmax of the last decode/generate step:
+ * the token id, or -1.  Synchronises the stream. */
+int32_t mk_last_argmax(mk_engine *e);
+
+/* Engine state I/O (checkpoint / resume and tests).  All buffers are device
+ * pointers in these layouts:
+ *   dn_state   [n_dn][dn_heads][dv][dk] float32
+ *   conv_state [n_dn][2*nh*dk + nh*dv][conv_k-1] float32
+ *   k_cache, v_cache [n_attn][kv_heads][pos][head_dim] bf16
+ * mk_set_state installs a state as if `pos` tokens had been consumed;
+ * mk_get_state copies the current one out (k/v caches may be NULL). */
+int mk_set_state(mk_engine *e, int pos, const float *dn_state,
+                 const float *conv_state, const void *k_cache,
+                 const void *v_cache);
+int mk_get_state(mk_engine *e, float *dn_state, float *conv_state,
+                 void *k_cache, void *v_cache);
+
+/* Residual stream after every layer for the last position processed by a
+ * decode, generate or prefill call: device float32 [n_layers][hidden]. */
+int mk_get_hidden(mk_engine *e, float *hidden_out);
+
+/* Launch statistics: number of kernels the engine launched so far. */
+int64_t mk_launch_count(const mk_engine *e);
+
+/* Debug: device-side wait limit in nanoseconds (default 2e9).  A grid
+ * barrier, pipeline or peer wait that exceeds it records MK_ERR_TIMEOUT and
+ * the kernel returns early.  `fail_barrier` >= 0 makes the next decode
+ * launch wait at that barrier for one arrival more than the grid provides,
+ * so the wait must run out (tests of the timeout path only). */
+int mk_debug_set_wait_limit(mk_engine *e, int64_t limit_ns, int fail_barrier);
+
+/* ------------------------------------------------------------------------
+ * Isolated gated delta-rule step (no engine).  One launch advances B
+ * sequences x heads of the recurrence by one token, in place:
+ *   S <- alpha S (I - beta k k^T) + beta v k^T ,   o = S q
+ * (Gated Delta Networks, the gated delta rule).
+ *   S     device float32 [B][heads][dv][dk]   state, read and written
+ *   q, k  device bf16    [B][heads][dk]       used as given (no renorm)
+ *   v     device bf16    [B][heads][dv]
+ *   alpha, beta device float32 [B][heads]
+ *   o     device float32 [B][heads][dv]
+ * dk == dv in {64, 128}.  `stream` is a cudaStream_t (may be NULL). */
+int mk_delta_step(float *S, const void *q, const void *k, const void *v,
+                  const float *alpha, const float *beta, float *o, int B,
+                  int heads, int dk, int dv, void *stream);
+
+/* Human-readable text of a status code. */
+const char *mk_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MK_H */

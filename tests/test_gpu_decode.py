@@ -1,0 +1,225 @@
+"""GPU parity of the single-launch decode engine against the fp64 oracle.
+
+Every call goes through the C ABI (libmk.so).  Teacher forcing: both sides
+consume the same token stream (the oracle's greedy choices), and each step's
+logits, per-layer residual stream and recurrent state are compared under the
+tolerances of tests/parity.py.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from attention_decode_megakernel_b200 import synth
+
+from parity import STATE_REL_L2, Tracker, rel_l2
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mk():
+    import attention_decode_megakernel_b200 as m
+    from attention_decode_megakernel_b200 import build
+    build.build()
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return m
+
+
+@pytest.fixture(scope="module")
+def big():
+    cfg = synth.hybrid_08b_config(max_ctx=1024)
+    return cfg, synth.make_weights(cfg)
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def _check_state(eng, orc, tol=STATE_REL_L2):
+    dn, conv, _, _ = eng.get_state()
+    odn, oconv = orc.get_state()
+    e_dn = rel_l2(_np(dn), odn)
+    e_conv = rel_l2(_np(conv), oconv)
+    assert e_dn <= tol, "DeltaNet state rel-L2 %.3e" % e_dn
+    assert e_conv <= tol, "conv state rel-L2 %.3e" % e_conv
+    return e_dn, e_conv
+
+
+def _teacher_forced(eng, orc, cfg, first_token, n_steps, tracker, check_hidden=True):
+    """n_steps decode steps; returns the tokens fed."""
+    logits = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
+    tok = int(first_token)
+    fed = []
+    for _ in range(n_steps):
+        eng.decode_step(tok, logits)
+        ref, ref_h = orc.step(tok, want_hidden=check_hidden)
+        eng.sync()
+        tracker.logits(_np(logits), ref)
+        if check_hidden:
+            tracker.hidden(_np(eng.get_hidden()), ref_h)
+        fed.append(tok)
+        tok = int(np.argmax(ref))
+    return fed
+
+
+def test_tiny_prompt_then_greedy_teacher_forced(mk):
+    cfg = synth.tiny_config(max_ctx=256)
+    w = synth.make_weights(cfg)
+    eng = mk.Engine(cfg, w)
+    orc = oracle.OracleModel(cfg, w)
+    tr = Tracker()
+    prompt = synth.make_tokens(cfg.vocab, 16)
+    logits = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
+    for t in prompt:
+        eng.decode_step(int(t), logits)
+        ref, ref_h = orc.step(int(t), want_hidden=True)
+        eng.sync()
+        tr.logits(_np(logits), ref)
+        tr.hidden(_np(eng.get_hidden()), ref_h)
+    _check_state(eng, orc)
+    _teacher_forced(eng, orc, cfg, int(np.argmax(ref)), 32, tr)
+    _check_state(eng, orc)
+    assert eng.position == 48 and orc.pos == 48
+    print(tr.finish())
+
+
+def test_tiny_prefill_matches_decode_loop(mk):
+    cfg = synth.tiny_config(max_ctx=256)
+    w = synth.make_weights(cfg)
+    prompt = synth.make_tokens(cfg.vocab, 40)
+    a = mk.Engine(cfg, w)
+    la = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
+    a.prefill(prompt, la)
+    orc = oracle.OracleModel(cfg, w)
+    for t in prompt:
+        ref, _ = orc.step(int(t))
+    a.sync()
+    tr = Tracker()
+    tr.logits(_np(la), ref)
+    _check_state(a, orc)
+
+
+def test_08b_decode_after_state_load(mk, big):
+    cfg, w = big
+    st = synth.make_engine_state(cfg, ctx=520)
+    eng = mk.Engine(cfg, w)
+    dev = {k: (torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v).cuda()
+               if isinstance(v, np.ndarray) else v) for k, v in st.items()}
+    eng.set_state(dev)
+    orc = oracle.OracleModel(cfg, w)
+    orc.set_state(st)
+    tr = Tracker()
+    _teacher_forced(eng, orc, cfg, 1234, 4, tr)
+    _check_state(eng, orc)
+    print(tr.finish())
+
+
+def test_08b_prompt_then_decode(mk, big):
+    cfg, w = big
+    eng = mk.Engine(cfg, w)
+    orc = oracle.OracleModel(cfg, w)
+    prompt = synth.make_tokens(cfg.vocab, 6)
+    logits = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
+    eng.prefill(prompt, logits)
+    for t in prompt:
+        ref, ref_h = orc.step(int(t), want_hidden=True)
+    eng.sync()
+    tr = Tracker()
+    tr.logits(_np(logits), ref)
+    tr.hidden(_np(eng.get_hidden()), ref_h)
+    _teacher_forced(eng, orc, cfg, int(np.argmax(ref)), 3, tr)
+    _check_state(eng, orc)
+    print(tr.finish())
+
+
+def test_generate_equals_decode_loop_bitwise(mk):
+    cfg = synth.tiny_config(max_ctx=256)
+    w = synth.make_weights(cfg)
+    prompt = synth.make_tokens(cfg.vocab, 8)
+    a, b = mk.Engine(cfg, w), mk.Engine(cfg, w)
+    a.prefill(prompt)
+    b.prefill(prompt)
+    n = 20
+    toks = torch.zeros(n, dtype=torch.int32, device="cuda")
+    a.generate(int(prompt[-1]) ^ 1, n, toks)
+    logits = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
+    tok, ref = int(prompt[-1]) ^ 1, []
+    for _ in range(n):
+        b.decode_step(tok, logits)
+        tok = int(torch.argmax(logits).item())
+        ref.append(tok)
+    assert _np(toks).tolist() == ref
+    assert a.last_argmax() == ref[-1]
+    sa, sb = a.get_state()[0], b.get_state()[0]
+    assert torch.equal(sa, sb)
+
+
+def test_verify_then_accept_equals_sequential_decode(mk):
+    cfg = synth.tiny_config(max_ctx=256)
+    w = synth.make_weights(cfg)
+    prompt = synth.make_tokens(cfg.vocab, 12)
+    drafts = synth.make_tokens(cfg.vocab, 5, seed=synth.SEED_DRAFTS)
+    a, b = mk.Engine(cfg, w), mk.Engine(cfg, w)
+    a.prefill(prompt)
+    b.prefill(prompt)
+    vl = torch.empty((5, cfg.vocab), dtype=torch.float32, device="cuda")
+    a.verify(drafts, vl)
+    assert a.position == 12
+    dl = torch.empty((5, cfg.vocab), dtype=torch.float32, device="cuda")
+    for j in range(5):
+        b.decode_step(int(drafts[j]), dl[j])
+    assert torch.equal(vl, dl)
+    # keep 2: state equals a fresh engine that decoded exactly 2 drafts
+    a.accept(2)
+    assert a.position == 14
+    c = mk.Engine(cfg, w)
+    c.prefill(prompt)
+    c.prefill(drafts[:2])
+    assert torch.equal(a.get_state()[0], c.get_state()[0])
+    assert torch.equal(a.get_state()[1], c.get_state()[1])
+    la, lc = torch.empty_like(dl[0]), torch.empty_like(dl[0])
+    a.decode_step(7, la)
+    c.decode_step(7, lc)
+    assert torch.equal(la, lc)
+
+
+def test_engine_errors(mk):
+    cfg = synth.tiny_config(max_ctx=4)
+    w = synth.make_weights(cfg)
+    eng = mk.Engine(cfg, w)
+    with pytest.raises(mk.MkError) as e:
+        eng.accept(1)
+    assert e.value.code == mk.MK_ERR_STATE
+    with pytest.raises(mk.MkError) as e:
+        eng.decode_step(cfg.vocab)
+    assert e.value.code == mk.MK_ERR_ARG
+    eng.prefill([1, 2, 3, 4])
+    with pytest.raises(mk.MkError) as e:
+        eng.decode_step(5)
+    assert e.value.code == mk.MK_ERR_CTX_OVERFLOW
+    eng.reset()
+    vl = torch.empty((9, cfg.vocab), dtype=torch.float32, device="cuda")
+    with pytest.raises(mk.MkError) as e:
+        eng.verify(list(range(9)), vl)
+    assert e.value.code == mk.MK_ERR_ARG
+
+
+def test_barrier_wait_limit_reports_timeout_and_recovers(mk):
+    """A barrier whose count can never be reached (one arrival more than the
+    grid has) must give up after the wait limit, report MK_ERR_TIMEOUT and
+    leave the context usable; mk_reset recovers the engine."""
+    cfg = synth.tiny_config(max_ctx=64)
+    w = synth.make_weights(cfg)
+    eng = mk.Engine(cfg, w)
+    eng.set_wait_limit(50_000_000, fail_barrier=3)  # 50 ms
+    eng.decode_step(3)
+    with pytest.raises(mk.MkError) as e:
+        eng.sync()
+    assert e.value.code == mk.MK_ERR_TIMEOUT
+    eng.reset()
+    eng.set_wait_limit(2_000_000_000, -1)
+    orc = oracle.OracleModel(cfg, w)
+    tr = Tracker()
+    _teacher_forced(eng, orc, cfg, 3, 3, tr)
