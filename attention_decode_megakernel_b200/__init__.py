@@ -227,8 +227,8 @@ class Engine:
     def launch_count(self) -> int:
         return int(lib().mk_launch_count(self._h))
 
-    def set_wait_limit(self, ns: int, fail_barrier: int = -1):
-        _check(lib().mk_debug_set_wait_limit(self._h, int(ns), int(fail_barrier)),
+    def set_wait_limit(self, ns: int, fail_phase: int = -1):
+        _check(lib().mk_debug_set_wait_limit(self._h, int(ns), int(fail_phase)),
                "mk_debug_set_wait_limit")
 
     def set_state(self, st: Dict):

@@ -4,25 +4,29 @@
 // layer with its MLP, final norm, tied LM head and greedy argmax) runs in ONE
 // cooperative launch of a persistent grid with one CTA per SM, as in the
 // launch post "OS Megakernel that match M5 Max Tok/w at 2x the Throughput on
-// RTX 3090" (kernel bullet list: whole forward pass in one dispatch,
-// cooperative grid sync instead of per-operation launches, bf16 weights with
-// fp32 accumulation, fused QKV + RoPE + causal softmax + output projection).
+// RTX 3090" (kernel bullet list: whole forward pass in one dispatch, no
+// per-operation launches, bf16 weights with fp32 accumulation, fused QKV +
+// RoPE + causal softmax + output projection).
 //
 // B200 structure (differs from the post's 3090 design):
 //  * Each CTA owns a balanced slice of every phase (rows of each matrix,
 //    rows of the recurrent state, a split of the KV cache).  The slices are
 //    known at launch, so one producer warp walks the CTA's whole per-token
-//    byte stream and keeps a 12 x 16 KB shared-memory ring full with bulk
-//    TMA copies (cp.async.bulk + mbarrier complete_tx).  It never waits on a
-//    grid barrier: weights, the previous token's state rows and the cached
-//    KV positions of the next phases keep streaming from HBM while the
-//    consumer warps wait for the rest of the grid.
-//  * Eight consumer warps turn each chunk into results: warp-per-row bf16
-//    GEMV against an fp32 activation vector held in registers, the gated
-//    delta-rule row update, split-K flash-decode attention with an
-//    online softmax and a last-CTA merge.  Phases that need the whole of the
-//    previous phase's output are separated by a grid barrier on a gpu-scope
-//    counter (release add / acquire poll), five per layer.
+//    byte stream and keeps a 6 x 32 KB shared-memory ring full with bulk TMA
+//    copies (cp.async.bulk + mbarrier complete_tx).  It never waits for
+//    other CTAs: weights, the previous token's state rows and cached KV
+//    positions of later phases keep streaming while the consumers wait.
+//  * Cross-CTA data travels as tagged words: every activation element another
+//    CTA needs is stored as one 8-byte word {fp32 value, 32-bit tag}, the tag
+//    naming the launch and the phase that produced it.  A consumer polls the
+//    words it needs until all tags match, so one L2 round trip both
+//    synchronises and delivers the vector; there is no grid barrier, no
+//    fence and no counter on the data path.  (The post's cooperative grid
+//    sync between layers is replaced by this data-driven wait.)
+//  * Seven consumer warps: bf16 GEMV rows (two per warp at a time) against an
+//    fp32 activation vector held in registers, the gated delta-rule row
+//    update, split-K flash-decode attention with an online softmax and a
+//    last-CTA merge, SwiGLU, the tied LM head with a grid argmax.
 //  * Every wait is bounded by %globaltimer; on expiry the kernel records
 //    MK_ERR_TIMEOUT, runs the rest of its schedule without work, lets its
 //    in-flight copies land and returns.
@@ -32,18 +36,25 @@
 
 namespace mk {
 
-constexpr int NCW = 8;                  // consumer warps
+constexpr int NCW = 7;                  // consumer warps (8 warps per CTA: 255 registers each)
 constexpr int NCT = NCW * 32;           // consumer threads
 constexpr int NTHR = NCT + 32;          // + producer warp
-constexpr int SLOT = 16384;             // ring slot bytes
-constexpr int NSLOT = 12;               // ring slots
+constexpr int SLOT = 32768;             // ring slot bytes
+constexpr int NSLOT = 6;                // ring slots
 constexpr int ATT_MIN_POS = 64;         // fewest positions per attention split
-constexpr int XREG_VEC = 8;             // activation vectors (8 floats) per lane held in registers
+constexpr int XRAW_MAX = 2048;          // largest hidden size (residual copy in shared memory)
+constexpr int UNION_FLOATS = 4096;      // activation vector | head cache | attention scratch
+constexpr int DN_HEADS_MAX = 4;         // heads one CTA's state rows may touch
+constexpr int DN_ROWS_MAX = 256;        // state rows of one CTA
+constexpr int CONV_ROWS_MAX = 256;      // in-projection rows of one CTA (conv staging)
+
+// words per consumer thread when NCT threads gather n tagged values
+constexpr int per_thread(int n) { return (n + NCT - 1) / NCT; }
 
 enum PhaseKind { PH_DN_IN, PH_DN_ST, PH_OUT, PH_Q, PH_K, PH_V, PH_ATT, PH_GU, PH_DOWN, PH_LM };
 
 struct StepArgs {
-  const DevModel* m;
+  DevModel m;         // the engine (by value: read through the constant bank)
   int pos;            // position of this token
   int token;          // input token when tok_src == 0
   int tok_src;        // 1: take the token from amax[amax_in]
@@ -52,8 +63,8 @@ struct StepArgs {
   float* logits;      // [V] (never NULL: scratch when the caller wants none)
   int32_t* tok_out;   // receives the argmax token (may be NULL)
   float* hidden;      // [n_layers][H] per-layer residual dump (may be NULL)
-  unsigned bar_base;  // grid-barrier counter value at launch
-  int fail_barrier;   // debug: barrier index that can never complete (-1 = none)
+  uint32_t seq;       // launch sequence number, 1 .. 2^23-1 (tag = seq << 8 | phase)
+  int fail_phase;     // debug: phase whose input tag can never match (-1 = none)
   long long wait_ns;  // bound of every device-side wait
 };
 
@@ -71,16 +82,12 @@ struct __align__(16) SmemTail {
 
 template <int DK, int HD, int GQ>
 struct Cfg {
-  static constexpr int EPL_S = DK / 32;  // state elements per lane
-  static constexpr int EPL_A = HD / 32;  // head elements per lane
-  static constexpr int GMAX = GQ;        // query heads per KV head
-  // union region (bytes): activation vector | DeltaNet head cache | attention scratch
-  static constexpr int XIN_FLOATS = 4096;
-  static constexpr int DNC_HEADS = 8;
-  static constexpr int ATT_FLOATS = GMAX * HD * 2 + 2 * HD + NCW * GMAX * 2;
-  static constexpr int UNION_FLOATS =
-      XIN_FLOATS > ATT_FLOATS ? XIN_FLOATS : ATT_FLOATS;
-  static constexpr size_t SMEM = size_t(NSLOT) * SLOT + sizeof(SmemTail) + UNION_FLOATS * 4 + 128;
+  static_assert(GQ * HD * 2 + 2 * HD + NCW * GQ * 2 <= UNION_FLOATS, "attention scratch");
+  static_assert(DN_HEADS_MAX * (2 * DK + 4) + 2 * DN_HEADS_MAX * DK + DN_ROWS_MAX +
+                    2 * DN_HEADS_MAX <= UNION_FLOATS,
+                "state-phase scratch");
+  static constexpr size_t SMEM =
+      size_t(NSLOT) * SLOT + sizeof(SmemTail) + (UNION_FLOATS + XRAW_MAX) * 4 + 128;
 };
 
 struct PD {                 // one CTA's share of one phase
@@ -199,84 +206,167 @@ __device__ __forceinline__ int layer_phases(const DevLayer& L, int* kinds) {
   kinds[0] = PH_DN_IN; kinds[1] = PH_DN_ST; kinds[2] = PH_OUT; kinds[3] = PH_GU; kinds[4] = PH_DOWN;
   return 5;
 }
-__device__ __forceinline__ bool has_grid_barrier(int kind) {
-  return !(kind == PH_Q || kind == PH_K || kind == PH_LM);
-}
 
 // ----------------------------------------------------------------------------
-// bounded waits
+// bounded waits and tagged words
 // ----------------------------------------------------------------------------
-__device__ __forceinline__ void record_error(const DevModel& M, int code) {
-  atomicCAS(M.err, 0, code);
-}
-
+__device__ __forceinline__ void record_error(int* err, int code) { atomicCAS(err, 0, code); }
 __device__ __forceinline__ bool aborted(SmemTail* t) { return *(volatile int*)&t->abort_flag != 0; }
+__device__ __forceinline__ void set_abort(SmemTail* t) { *(volatile int*)&t->abort_flag = 1; }
 
-// Returns false (and leaves the CTA in abort mode) when the wait gave up.
+// Give up a wait that started at `start`: true (and abort mode) once the CTA
+// aborted or the limit passed.
+__device__ __forceinline__ bool give_up(SmemTail* t, int* err, uint64_t start,
+                                        long long wait_ns) {
+  if (aborted(t)) return true;
+  if (global_ns() - start > uint64_t(wait_ns)) {
+    record_error(err, MK_ERR_TIMEOUT);
+    set_abort(t);
+    return true;
+  }
+  return false;
+}
+
+// Wait on a ring mbarrier phase; false (and abort mode) when the wait gave up.
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, SmemTail* t,
-                                             const DevModel& M, long long wait_ns) {
+                                             int* err, long long wait_ns) {
   if (aborted(t)) return false;
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t start = global_ns();
+  const uint64_t start = global_ns();
   for (int it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 31) == 0) {
-      if (*(volatile int*)&t->abort_flag) return false;
-      if (global_ns() - start > uint64_t(wait_ns)) {
-        record_error(M, MK_ERR_TIMEOUT);
-        *(volatile int*)&t->abort_flag = 1;
-        return false;
-      }
-    }
+    if ((it & 31) == 0 && give_up(t, err, start, wait_ns)) return false;
   }
 }
 
-// Grid barrier number `k` of this launch (one thread per CTA).
-__device__ __forceinline__ bool grid_barrier(const DevModel& M, const StepArgs& a, int k,
-                                             SmemTail* t) {
+__device__ __forceinline__ uint32_t make_tag(uint32_t seq, int phase) {
+  return (seq << 8) | uint32_t(phase & 0xFF);
+}
+__device__ __forceinline__ void ll_put(unsigned long long* p, float v, uint32_t tag) {
+  unsigned long long w = (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(v);
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+__device__ __forceinline__ unsigned long long ll_get(const unsigned long long* p) {
+  unsigned long long w;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+  return w;
+}
+
+// Consumer threads cooperatively fetch n tagged values into shared memory
+// (dst[i] = value of src[i]) once every tag equals `tag`.  Thread tid handles
+// i = tid + j*NCT; all its words are in flight at once.  Returns false on
+// timeout / abort (per thread; callers agree through named_sync_or).
+template <int MAXK>
+__device__ __forceinline__ bool ll_gather(float* dst, const unsigned long long* src, int n,
+                                          uint32_t tag, SmemTail* t, int* err,
+                                          long long wait_ns, int tid) {
   if (aborted(t)) return false;
-  __threadfence();
-  red_add_release_gpu(M.bar, 1u);
-  unsigned target = a.bar_base + unsigned(k + 1) * unsigned(M.ncta);
-  if (k == a.fail_barrier) target += 1u;  // debug: one arrival more than exists
-  uint64_t start = global_ns();
+  unsigned long long w[MAXK];
+  uint64_t start = 0;
   for (int it = 0;; ++it) {
-    unsigned v = ld_acquire_gpu(M.bar);
-    if (int(v - target) >= 0) return true;
-    if ((it & 15) == 15) {
-      if (ld_relaxed_gpu(M.err) != 0) {
-        *(volatile int*)&t->abort_flag = 1;
-        return false;
-      }
-      if (global_ns() - start > uint64_t(a.wait_ns)) {
-        record_error(M, MK_ERR_TIMEOUT);
-        *(volatile int*)&t->abort_flag = 1;
-        return false;
-      }
+#pragma unroll
+    for (int j = 0; j < MAXK; ++j) {
+      const int i = tid + j * NCT;
+      unsigned long long v = static_cast<unsigned long long>(tag) << 32;
+      if (i < n) v = ll_get(src + i);
+      w[j] = v;
     }
+    bool stale = false;
+#pragma unroll
+    for (int j = 0; j < MAXK; ++j) stale |= uint32_t(w[j] >> 32) != tag;
+    if (!stale) break;
+    if (it == 0) start = global_ns();
+    else if ((it & 7) == 0 && give_up(t, err, start, wait_ns)) return false;
+  }
+#pragma unroll
+  for (int j = 0; j < MAXK; ++j) {
+    const int i = tid + j * NCT;
+    if (i < n) dst[i] = __uint_as_float(uint32_t(w[j]));
+  }
+  return true;
+}
+
+// One tagged value by one thread.
+__device__ __forceinline__ bool ll_wait1(float& out, const unsigned long long* src, uint32_t tag,
+                                         SmemTail* t, int* err, long long wait_ns) {
+  if (aborted(t)) return false;
+  uint64_t start = 0;
+  for (int it = 0;; ++it) {
+    const unsigned long long w = ll_get(src);
+    if (uint32_t(w >> 32) == tag) {
+      out = __uint_as_float(uint32_t(w));
+      return true;
+    }
+    if (it == 0) start = global_ns();
+    else if ((it & 7) == 0 && give_up(t, err, start, wait_ns)) return false;
   }
 }
 
-// ----------------------------------------------------------------------------
-// GEMV helpers (warp per row)
-// ----------------------------------------------------------------------------
-__device__ __forceinline__ void load_xregs(float (&xr)[XREG_VEC][8], const float* xin, int nvec,
-                                           int lane) {
+// Gather several tagged ranges at once (one polling round trip for all):
+// segment i copies n values from src to dst (shared memory).
+struct LLSeg {
+  const unsigned long long* src;
+  float* dst;
+  int n;
+  uint32_t tag;  // the tag every word of this segment must carry
+};
+
+template <int MAXK, int NSEG>
+__device__ __forceinline__ bool ll_gather_segs(const LLSeg (&sg)[NSEG], SmemTail* t, int* err,
+                                               long long wait_ns, int tid) {
+  if (aborted(t)) return false;
+  const unsigned long long* src[MAXK];
+  float* dst[MAXK];
+  uint32_t tg[MAXK];
+  int total = 0;
 #pragma unroll
-  for (int v = 0; v < XREG_VEC; ++v) {
-    int idx = v * 32 + lane;
-    if (idx < nvec) {
-      float4 p = reinterpret_cast<const float4*>(xin)[idx * 2];
-      float4 q = reinterpret_cast<const float4*>(xin)[idx * 2 + 1];
-      xr[v][0] = p.x; xr[v][1] = p.y; xr[v][2] = p.z; xr[v][3] = p.w;
-      xr[v][4] = q.x; xr[v][5] = q.y; xr[v][6] = q.z; xr[v][7] = q.w;
-    } else {
+  for (int q = 0; q < NSEG; ++q) total += sg[q].n;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) xr[v][e] = 0.f;
+  for (int j = 0; j < MAXK; ++j) {
+    int i = tid + j * NCT;
+    src[j] = nullptr;
+    dst[j] = nullptr;
+    tg[j] = 0;
+    if (i < total) {
+#pragma unroll
+      for (int q = 0; q < NSEG; ++q) {
+        if (i >= 0 && i < sg[q].n) {
+          src[j] = sg[q].src + i;
+          dst[j] = sg[q].dst + i;
+          tg[j] = sg[q].tag;
+        }
+        i -= sg[q].n;
+      }
     }
   }
+  unsigned long long w[MAXK];
+  uint64_t start = 0;
+  for (int it = 0;; ++it) {
+#pragma unroll
+    for (int j = 0; j < MAXK; ++j) {
+      unsigned long long v = static_cast<unsigned long long>(tg[j]) << 32;
+      if (src[j]) v = ll_get(src[j]);
+      w[j] = v;
+    }
+    bool stale = false;
+#pragma unroll
+    for (int j = 0; j < MAXK; ++j) stale |= uint32_t(w[j] >> 32) != tg[j];
+    if (!stale) break;
+    if (it == 0) start = global_ns();
+    else if ((it & 7) == 0 && give_up(t, err, start, wait_ns)) return false;
+  }
+#pragma unroll
+  for (int j = 0; j < MAXK; ++j)
+    if (dst[j]) *dst[j] = __uint_as_float(uint32_t(w[j]));
+  return true;
 }
 
+// ----------------------------------------------------------------------------
+// GEMV helpers (warp per row).  Lane l owns 16-byte weight vectors
+// v*32 + l of a row (8 bf16 each) and the matching 8 activation floats.  The
+// vector count per lane NV is a compile-time constant: a runtime bound on the
+// unrolled loop costs more than the arithmetic.
+// ----------------------------------------------------------------------------
 __device__ __forceinline__ void fma8(const uint4 w, const float* x, float& a0, float& a1,
                                      float& a2, float& a3) {
   a0 = fmaf(bf_lo(w.x), x[0], a0);
@@ -289,45 +379,226 @@ __device__ __forceinline__ void fma8(const uint4 w, const float* x, float& a0, f
   a3 = fmaf(bf_hi(w.w), x[7], a3);
 }
 
-// Partial dot of one bf16 row (nvec 16-byte vectors in shared memory) with
-// the register-resident activation; the caller reduces over the warp.
-__device__ __forceinline__ float row_dot_regs(const uint4* w, const float (&xr)[XREG_VEC][8],
-                                              int nvec, int lane) {
+// PRED: the row has fewer than 32 vectors (small models), lanes past nvec idle.
+template <int NV, bool PRED>
+__device__ __forceinline__ void load_x(float (&xr)[NV][8], const float* xs, int nvec, int lane) {
+#pragma unroll
+  for (int v = 0; v < NV; ++v) {
+    const int idx = v * 32 + lane;
+    if (!PRED || idx < nvec) {
+      const float4 p = reinterpret_cast<const float4*>(xs)[idx * 2];
+      const float4 q = reinterpret_cast<const float4*>(xs)[idx * 2 + 1];
+      xr[v][0] = p.x; xr[v][1] = p.y; xr[v][2] = p.z; xr[v][3] = p.w;
+      xr[v][4] = q.x; xr[v][5] = q.y; xr[v][6] = q.z; xr[v][7] = q.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) xr[v][e] = 0.f;
+    }
+  }
+}
+
+template <int NV, bool PRED>
+__device__ __forceinline__ float dot_x(const unsigned char* row, const float (&xr)[NV][8],
+                                       int nvec, int lane) {
+  const uint4* w = reinterpret_cast<const uint4*>(row);
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-  for (int v = 0; v < XREG_VEC; ++v) {
-    int idx = v * 32 + lane;
-    if (idx < nvec) fma8(w[idx], xr[v], a0, a1, a2, a3);
+  for (int v = 0; v < NV; ++v) {
+    const int idx = v * 32 + lane;
+    if (!PRED || idx < nvec) fma8(w[idx], xr[v], a0, a1, a2, a3);
   }
   return (a0 + a1) + (a2 + a3);
 }
 
-// Same with the activation read from shared memory (long rows).
-__device__ __forceinline__ float row_dot_smem(const uint4* w, const float* xin, int nvec,
-                                              int lane) {
+__device__ __forceinline__ void fma8_xs(const uint4 w, const float* xs, int idx, float& a0,
+                                        float& a1, float& a2, float& a3) {
+  float x[8];
+  const float4 p = reinterpret_cast<const float4*>(xs)[idx * 2];
+  const float4 q = reinterpret_cast<const float4*>(xs)[idx * 2 + 1];
+  x[0] = p.x; x[1] = p.y; x[2] = p.z; x[3] = p.w;
+  x[4] = q.x; x[5] = q.y; x[6] = q.z; x[7] = q.w;
+  fma8(w, x, a0, a1, a2, a3);
+}
+
+// Activation read from shared memory (rows too long for registers).  NV > 0:
+// exactly NV vectors per lane; NV == 0: any length (runtime loop).
+template <int NV>
+__device__ __forceinline__ float dot_xs(const unsigned char* row, const float* xs, int nvec,
+                                        int lane) {
+  const uint4* w = reinterpret_cast<const uint4*>(row);
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  for (int idx = lane; idx < nvec; idx += 32) {
-    float x[8];
-    float4 p = reinterpret_cast<const float4*>(xin)[idx * 2];
-    float4 q = reinterpret_cast<const float4*>(xin)[idx * 2 + 1];
-    x[0] = p.x; x[1] = p.y; x[2] = p.z; x[3] = p.w;
-    x[4] = q.x; x[5] = q.y; x[6] = q.z; x[7] = q.w;
-    fma8(w[idx], x, a0, a1, a2, a3);
+  if constexpr (NV > 0) {
+#pragma unroll
+    for (int v = 0; v < NV; ++v) fma8_xs(w[v * 32 + lane], xs, v * 32 + lane, a0, a1, a2, a3);
+  } else {
+    for (int idx = lane; idx < nvec; idx += 32) fma8_xs(w[idx], xs, idx, a0, a1, a2, a3);
   }
   return (a0 + a1) + (a2 + a3);
 }
 
+// ---- matrix phases ------------------------------------------------------------
+// One out-of-line routine serves every matrix phase, so the hot loop exists
+// once in the instruction stream (a phase switch then finds it cached); the
+// epilogue is a small runtime switch.
+enum EpiKind { EPI_STORE, EPI_RESID, EPI_INPROJ, EPI_SWIGLU, EPI_LOGITS };
+
+struct GemvJob {
+  PD d;
+  int epi;                   // EpiKind
+  int shape;                 // GemvShape of the row length
+  unsigned long long* dst;   // tagged destination, indexed by row
+  const float* xraw;         // EPI_RESID: residual before the update (shared memory)
+  float* hidden;             // EPI_RESID: optional per-layer dump
+  const float4* conv_s;      // EPI_INPROJ: conv history rows staged in shared memory
+  const uint2* conv_taps;    // EPI_INPROJ: conv taps rows staged in shared memory
+  float4* conv_out;          // EPI_INPROJ: the layer's conv history in global memory
+  int ch;                    // EPI_INPROJ: conv channels (rows below ch get the conv)
+  float* logits;             // EPI_LOGITS
+  uint32_t tag;
+};
+
+__device__ __forceinline__ void gemv_epilogue(const GemvJob& j, int row, float y, float y2,
+                                              float& best_v, int& best_i) {
+  switch (j.epi) {
+    case EPI_STORE:
+      ll_put(j.dst + row, y, j.tag);
+      break;
+    case EPI_RESID: {
+      const float v = j.xraw[row] + y;
+      ll_put(j.dst + row, v, j.tag);
+      if (j.hidden) j.hidden[row] = v;
+      break;
+    }
+    case EPI_INPROJ:
+      if (row < j.ch) {
+        // taps (u_{t-3}, u_{t-2}, u_{t-1}, u_t); shift the history by one
+        const float4 s = j.conv_s[row - j.d.r0];
+        const uint2 wc = j.conv_taps[row - j.d.r0];
+        const float c =
+            bf_lo(wc.x) * s.x + bf_hi(wc.x) * s.y + bf_lo(wc.y) * s.z + bf_hi(wc.y) * y;
+        j.conv_out[row] = make_float4(s.y, s.z, y, 0.f);
+        ll_put(j.dst + row, siluf_(c), j.tag);
+      } else {
+        ll_put(j.dst + row, y, j.tag);
+      }
+      break;
+    case EPI_SWIGLU:
+      ll_put(j.dst + row, siluf_(y) * y2, j.tag);
+      break;
+    case EPI_LOGITS:
+      j.logits[row] = y;
+      if (y > best_v || (y == best_v && row < best_i)) {
+        best_v = y;
+        best_i = row;
+      }
+      break;
+  }
+}
+
+// Walk the CTA's chunks of one matrix phase.  Each warp takes its rows of a
+// chunk two at a time (independent reductions overlap); for EPI_SWIGLU the
+// pair is a gate row (plane 0) and the matching up row (plane 1).  NV/PRED/XS
+// select the activation layout (see dot_x / dot_xs).  Returns the chunk
+// counter after the phase.
+template <int NV, bool PRED, bool XS>
+__device__ __forceinline__ uint32_t gemv_core(const GemvJob& j, uint32_t g, unsigned char* ring,
+                                              SmemTail* t, int* err, long long wait_ns,
+                                              const float* xs) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const PD& d = j.d;
+  const int nvec = int(d.row_bytes / 16);
+  const bool swiglu = j.epi == EPI_SWIGLU;
+  constexpr int NR = XS ? 1 : NV;
+  float xr[NR][8];
+  if constexpr (!XS) load_x<NV, PRED>(xr, xs, nvec, lane);
+  float best_v = -INFINITY;
+  int best_i = 0x7FFFFFFF;
+  int local = 0;
+#pragma unroll 1
+  for (int r = d.r0; r < d.r0 + d.n; r += d.rpc, ++g, local += d.rpc) {
+    const int slot = int(g % NSLOT);
+    if (bounded_wait(&t->full[slot], (g / NSLOT) & 1, t, err, wait_ns)) {
+      const int nr = min(d.rpc, d.r0 + d.n - r);
+      const unsigned char* base = ring + size_t(slot) * SLOT;
+      const int step = swiglu ? NCW : 2 * NCW;
+#pragma unroll 1
+      for (int i = (warp - (local % NCW) + NCW) % NCW; i < nr; i += step) {
+        // rows a and b: (i, i + NCW) of plane 0, or (i of plane 0, i of plane 1)
+        const int ib = swiglu ? i : i + NCW;
+        const bool hb = swiglu || ib < nr;
+        const unsigned char* ra = base + size_t(i) * d.row_bytes;
+        const unsigned char* rb = base + size_t(swiglu ? d.rpc + i : ib) * d.row_bytes;
+        float pa, pb = 0.f;
+        if constexpr (XS) {
+          pa = dot_xs<NV>(ra, xs, nvec, lane);
+          if (hb) pb = dot_xs<NV>(rb, xs, nvec, lane);
+        } else {
+          pa = dot_x<NV, PRED>(ra, xr, nvec, lane);
+          if (hb) pb = dot_x<NV, PRED>(rb, xr, nvec, lane);
+        }
+        pa = warp_sum(pa);
+        pb = warp_sum(pb);
+        if (lane == 0) {
+          if (swiglu) {
+            gemv_epilogue(j, r + i, pa, pb, best_v, best_i);
+          } else {
+            gemv_epilogue(j, r + i, pa, 0.f, best_v, best_i);
+            if (hb) gemv_epilogue(j, r + ib, pb, 0.f, best_v, best_i);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&t->empty[slot]);
+  }
+  if (j.epi == EPI_LOGITS && lane == 0 && best_i != 0x7FFFFFFF)
+    atomicMax(&t->best, pack_argmax(best_v, best_i));
+  return g;
+}
+
+// Activation layouts the kernel instantiates (chosen from the row length K,
+// a multiple of 8): fewer than 32 vectors (predicated), 1/2/3/4/8 vectors per
+// lane in registers, 14 per lane from shared memory, anything else from
+// shared memory with a runtime loop.
+enum GemvShape { GS_PRED1 = 0, GS_R1, GS_R2, GS_R3, GS_R4, GS_R8, GS_S14, GS_SANY };
+
+__host__ __device__ constexpr int gemv_shape(int K) {
+  return (K / 8) < 32        ? GS_PRED1
+         : (K / 8) % 32 != 0 ? GS_SANY
+         : (K / 256) == 1    ? GS_R1
+         : (K / 256) == 2    ? GS_R2
+         : (K / 256) == 3    ? GS_R3
+         : (K / 256) == 4    ? GS_R4
+         : (K / 256) == 8    ? GS_R8
+         : (K / 256) == 14   ? GS_S14
+                             : GS_SANY;
+}
+
+__device__ __forceinline__ uint32_t gemv_dispatch(const GemvJob& j, uint32_t g,
+                                                  unsigned char* ring, SmemTail* t, int* err,
+                                                  long long wait_ns, const float* xs) {
+  switch (j.shape) {
+    case GS_PRED1: return gemv_core<1, true, false>(j, g, ring, t, err, wait_ns, xs);
+    case GS_R1: return gemv_core<1, false, false>(j, g, ring, t, err, wait_ns, xs);
+    case GS_R2: return gemv_core<2, false, false>(j, g, ring, t, err, wait_ns, xs);
+    case GS_R3: return gemv_core<3, false, false>(j, g, ring, t, err, wait_ns, xs);
+    case GS_R4: return gemv_core<4, false, false>(j, g, ring, t, err, wait_ns, xs);
+    case GS_R8: return gemv_core<8, false, false>(j, g, ring, t, err, wait_ns, xs);
+    case GS_S14: return gemv_core<14, false, true>(j, g, ring, t, err, wait_ns, xs);
+    default: return gemv_core<0, false, true>(j, g, ring, t, err, wait_ns, xs);
+  }
+}
+
 // ----------------------------------------------------------------------------
-// consumer pre-phase builders (all NCT consumer threads)
+// RMSNorm of the vector already in `xin` (all NCT consumer threads):
+// xin = xin * rsqrt(mean(xin^2) + eps) * gain, keeping the raw copy in xraw.
 // ----------------------------------------------------------------------------
-// xin = RMSNorm(src) * gain; src is the fp32 residual (gpu-coherent loads) or,
-// for the first layer, the bf16 embedding row of the token.
-__device__ void build_rmsnorm(float* xin, const float* src, const uint16_t* emb_row,
-                              const uint16_t* gain, int H, float eps, SmemTail* t, int tid) {
+__device__ __forceinline__ void rmsnorm_inplace(float* xin, float* xraw, const uint16_t* gain,
+                                                int H, float eps, SmemTail* t, int tid) {
   float ss = 0.f;
   for (int i = tid; i < H; i += NCT) {
-    float v = emb_row ? bf2f(emb_row[i]) : __ldcg(src + i);
-    xin[i] = v;
+    const float v = xin[i];
+    if (xraw) xraw[i] = v;
     ss = fmaf(v, v, ss);
   }
   ss = warp_sum(ss);
@@ -336,57 +607,20 @@ __device__ void build_rmsnorm(float* xin, const float* src, const uint16_t* emb_
   float tot = 0.f;
 #pragma unroll
   for (int w = 0; w < NCW; ++w) tot += t->red[w];
-  float inv = 1.0f / sqrtf(tot / float(H) + eps);
+  const float inv = 1.0f / sqrtf(tot / float(H) + eps);
   for (int i = tid; i < H; i += NCT) xin[i] = xin[i] * inv * bf2f(gain[i]);
   named_sync(1, NCT);
 }
 
-__device__ void build_copy(float* xin, const float* src, int n, int tid) {
-  for (int i = tid; i < n; i += NCT) xin[i] = __ldcg(src + i);
-  named_sync(1, NCT);
-}
-
-// xin[h*dv+i] = RMSNorm_dv(o_h)_i * out_norm_i * SiLU(z_h,i): the gated
-// output norm of the DeltaNet layer (warp per head).
-template <int DK>
-__device__ void build_gated_norm(float* xin, const DevModel& M, const DevLayer& L, int tid) {
-  constexpr int EPL = DK / 32;  // dv == dk
-  int warp = tid >> 5, lane = tid & 31;
-  const float* z = M.inp + M.ch;
-  for (int h = warp; h < M.nh; h += NCW) {
-    float o[EPL];
-    float ss = 0.f;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      o[e] = __ldcg(M.dno + h * M.dv + lane * EPL + e);
-      ss = fmaf(o[e], o[e], ss);
-    }
-    ss = warp_sum(ss);
-    float inv = 1.0f / sqrtf(ss / float(M.dv) + M.eps);
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      int i = lane * EPL + e;
-      float zz = __ldcg(z + h * M.dv + i);
-      xin[h * M.dv + i] = o[e] * inv * bf2f(L.out_norm[i]) * siluf_(zz);
-    }
-  }
-  named_sync(1, NCT);
-}
-
-// ----------------------------------------------------------------------------
-// consumer chunk loop: wait for each chunk of the CTA's share of a phase,
-// hand this warp's rows to `fn(row, plane0_row, plane1_row)`, release the slot
-// ----------------------------------------------------------------------------
-// (A macro rather than a function taking a lambda: the body must be inlined
-// so that register-resident activations and accumulators stay in registers.)
-// Uses the enclosing scope's M, a, t, ring, g, warp, lane; the body sees
-// `row`, `p0` (plane-0 row in shared memory) and `p1` (plane-1 row).
+// Chunk loop for the non-GEMV phases (state rows, KV positions): the body
+// sees `row`, `p0` (plane-0 row in shared memory) and `p1` (plane-1 row).
+// (A macro: the body must be inlined so register arrays stay in registers.)
 #define MK_CHUNK_LOOP(d, ...)                                                          \
   do {                                                                                 \
     int local_ = 0;                                                                    \
     for (int r_ = (d).r0; r_ < (d).r0 + (d).n; r_ += (d).rpc, ++g, local_ += (d).rpc) { \
       const int slot_ = int(g % NSLOT);                                                \
-      const bool ok_ = bounded_wait(&t->full[slot_], (g / NSLOT) & 1, t, M, a.wait_ns); \
+      const bool ok_ = bounded_wait(&t->full[slot_], (g / NSLOT) & 1, t, M.err, a.wait_ns); \
       if (ok_) {                                                                       \
         const int nr_ = min((d).rpc, (d).r0 + (d).n - r_);                             \
         const unsigned char* base_ = ring + size_t(slot_) * SLOT;                      \
@@ -410,21 +644,38 @@ template <int DK>
 __device__ __forceinline__ void dn_state_phase(const DevModel& M, const StepArgs& a,
                                                const DevLayer& L, const PD& d, uint32_t& g,
                                                unsigned char* ring, SmemTail* t, float* uni,
-                                               bool dry, int tid, int warp, int lane) {
+                                               uint32_t tag_in, uint32_t tag_out, bool dry,
+                                               int tid, int warp, int lane) {
   constexpr int EPL = DK / 32;
   constexpr int stride = 2 * DK + 4;  // head cache: [q(dk) | k(dk) | beta, alpha, k.q, -]
-  int h_first = 0;
+  const int h_first = d.n > 0 ? d.r0 / M.dv : 0;
+  const int n_heads = d.n > 0 ? (d.r0 + d.n - 1) / M.dv - h_first + 1 : 0;
+  // staging: raw q, k of the touched heads, v of this CTA's rows, b and a
+  float* sq_raw = uni + DN_HEADS_MAX * stride;   // [n_heads][DK]
+  float* sk_raw = sq_raw + DN_HEADS_MAX * DK;    // [n_heads][DK]
+  float* vrow = sk_raw + DN_HEADS_MAX * DK;      // [d.n]
+  float* sba = vrow + DN_ROWS_MAX;               // [2][n_heads]
+  bool ok = true;
   if (!dry && d.n > 0) {
-    h_first = d.r0 / M.dv;
-    const int h_last = (d.r0 + d.n - 1) / M.dv;
-    for (int hh = warp; hh <= h_last - h_first; hh += NCW) {
+    const LLSeg sg[5] = {
+        {M.inp_ll + h_first * DK, sq_raw, n_heads * DK, tag_in},
+        {M.inp_ll + M.nh * DK + h_first * DK, sk_raw, n_heads * DK, tag_in},
+        {M.inp_ll + 2 * M.nh * DK + d.r0, vrow, d.n, tag_in},
+        {M.inp_ll + M.ch + M.nh * M.dv + h_first, sba, n_heads, tag_in},
+        {M.inp_ll + M.ch + M.nh * M.dv + M.nh + h_first, sba + DN_HEADS_MAX, n_heads, tag_in}};
+    ok = ll_gather_segs<per_thread(2 * DN_HEADS_MAX * DK + DN_ROWS_MAX + 2 * DN_HEADS_MAX), 5>(
+        sg, t, M.err, a.wait_ns, tid);
+  }
+  const bool bad = named_sync_or(1, NCT, !ok);
+  if (!dry && !bad) {
+    for (int hh = warp; hh < n_heads; hh += NCW) {
       const int h = h_first + hh;
       float qv[EPL], kv[EPL];
       float sq = 0.f, sk = 0.f;
 #pragma unroll
       for (int e = 0; e < EPL; ++e) {
-        qv[e] = __ldcg(M.inp + h * DK + lane * EPL + e);
-        kv[e] = __ldcg(M.inp + M.nh * DK + h * DK + lane * EPL + e);
+        qv[e] = sq_raw[hh * DK + lane * EPL + e];
+        kv[e] = sk_raw[hh * DK + lane * EPL + e];
         sq = fmaf(qv[e], qv[e], sq);
         sk = fmaf(kv[e], kv[e], sk);
       }
@@ -444,18 +695,18 @@ __device__ __forceinline__ void dn_state_phase(const DevModel& M, const StepArgs
       }
       kq = warp_sum(kq);
       if (lane == 0) {
-        const float b = __ldcg(M.inp + M.ch + M.nh * M.dv + h);
-        const float aa = __ldcg(M.inp + M.ch + M.nh * M.dv + M.nh + h);
-        uni[hh * stride + 2 * DK + 0] = sigmoidf_(b);                                   // beta
-        uni[hh * stride + 2 * DK + 1] = expf(-expf(L.A_log[h]) * softplusf_(aa + L.dt_bias[h]));  // alpha
+        const float b = sba[hh], aa = sba[DN_HEADS_MAX + hh];
+        uni[hh * stride + 2 * DK + 0] = sigmoidf_(b);  // beta
+        uni[hh * stride + 2 * DK + 1] =
+            expf(-expf(L.A_log[h]) * softplusf_(aa + L.dt_bias[h]));  // alpha
         uni[hh * stride + 2 * DK + 2] = kq;
       }
     }
   }
   named_sync(1, NCT);
   float* st = M.dn_state[a.st_buf] + size_t(L.sub) * M.nh * M.dv * DK;
-  MK_CHUNK_LOOP(d, 
-    const int h = row / M.dv, iv = row % M.dv;
+  MK_CHUNK_LOOP(d, {
+    const int h = row / M.dv;
     const float* hc = uni + (h - h_first) * stride;
     const float* sr = reinterpret_cast<const float*>(p0) + lane * EPL;
     float sv[EPL], kv[EPL];
@@ -470,8 +721,7 @@ __device__ __forceinline__ void dn_state_phase(const DevModel& M, const StepArgs
     s_k = warp_sum(s_k);
     s_q = warp_sum(s_q);
     const float beta = hc[2 * DK], alpha = hc[2 * DK + 1], kq = hc[2 * DK + 2];
-    const float vi = __ldcg(M.inp + 2 * M.nh * DK + h * M.dv + iv);
-    const float u = beta * (vi - alpha * s_k);  // S' = alpha S + u k^T
+    const float u = beta * (vrow[row - d.r0] - alpha * s_k);  // S' = alpha S + u k^T
     float* dst = st + size_t(row) * DK + lane * EPL;
     if constexpr (EPL == 4) {
       *reinterpret_cast<float4*>(dst) =
@@ -481,8 +731,8 @@ __device__ __forceinline__ void dn_state_phase(const DevModel& M, const StepArgs
 #pragma unroll
       for (int e = 0; e < EPL; ++e) dst[e] = fmaf(alpha, sv[e], u * kv[e]);
     }
-    if (lane == 0) M.dno[row] = fmaf(alpha, s_q, u * kq);  // o_i = S'_i . q
-  );
+    if (lane == 0) ll_put(M.dno_ll + row, fmaf(alpha, s_q, u * kq), tag_out);  // o_i = S'_i.q
+  });
 }
 
 // One key/value row into a warp's online-softmax state for G query heads
@@ -514,7 +764,9 @@ template <int HD, int GQ>
 __device__ __forceinline__ void attention_phase(const DevModel& M, const StepArgs& a,
                                                 const DevLayer& L, const PD& d, uint32_t& g,
                                                 unsigned char* ring, SmemTail* t, float* uni,
-                                                bool dry, int tid, int warp, int lane) {
+                                                uint32_t tag_q, uint32_t tag_k, uint32_t tag_v,
+                                                uint32_t tag_out, bool dry, int tid, int warp,
+                                                int lane) {
   constexpr int EPL = HD / 32;
   constexpr int G = GQ;
   float* att_q = uni;                   // [G][HD] rotated queries
@@ -525,24 +777,36 @@ __device__ __forceinline__ void attention_phase(const DevModel& M, const StepArg
   const bool unit = d.unit_g >= 0;
   const bool last = unit && d.unit_s == d.S - 1;
   const int gidx = d.unit_g;
+  const int half = HD / 2;
+  bool ok = true;
   if (unit && !dry) {
-    const int half = HD / 2;
+    // raw q of the group's heads (staged in att_acc) and, for the split that
+    // owns the new position, its raw k and v: one polling round
+    const LLSeg sg[3] = {
+        {M.qkv_ll + gidx * G * HD, att_acc, G * HD, tag_q},
+        {M.qkv_ll + M.nq * HD + gidx * HD, att_kn, last ? HD : 0, tag_k},
+        {M.qkv_ll + (M.nq + M.nkv) * HD + gidx * HD, att_vn, last ? HD : 0, tag_v}};
+    ok = ll_gather_segs<per_thread(GQ * HD + 2 * HD), 3>(sg, t, M.err, a.wait_ns, tid);
+  }
+  const bool bad = named_sync_or(1, NCT, !ok);
+  const bool work = unit && !dry && !bad;
+  if (work) {
     for (int i = tid; i < G * half; i += NCT) {
       const int j = i / half, c = i % half;
-      const float* qh = M.qkv + (gidx * G + j) * HD;
-      const float x0 = __ldcg(qh + c), x1 = __ldcg(qh + c + half);
+      const float x0 = att_acc[j * HD + c], x1 = att_acc[j * HD + c + half];
       const float cs = t->rope_cos[c], sn = t->rope_sin[c];
       att_q[j * HD + c] = x0 * cs - x1 * sn;
       att_q[j * HD + c + half] = x1 * cs + x0 * sn;
     }
+  }
+  named_sync(1, NCT);
+  if (work) {
     for (int i = tid; i < G * HD; i += NCT) att_acc[i] = 0.f;
     if (last) {
       // RoPE the new key, store K/V at `pos` in bf16, keep the rounded values
-      const float* kr = M.qkv + M.nq * HD + gidx * HD;
-      const float* vr = M.qkv + (M.nq + M.nkv) * HD + gidx * HD;
       const size_t cofs = ((size_t(L.sub) * M.nkv + gidx) * M.max_ctx + a.pos) * HD;
       for (int c = tid; c < half; c += NCT) {
-        const float x0 = __ldcg(kr + c), x1 = __ldcg(kr + c + half);
+        const float x0 = att_kn[c], x1 = att_kn[c + half];
         const float cs = t->rope_cos[c], sn = t->rope_sin[c];
         const uint16_t b0 = f2bf(x0 * cs - x1 * sn), b1 = f2bf(x1 * cs + x0 * sn);
         M.kc[cofs + c] = b0;
@@ -551,7 +815,7 @@ __device__ __forceinline__ void attention_phase(const DevModel& M, const StepArg
         att_kn[c + half] = bf2f(b1);
       }
       for (int c = tid; c < HD; c += NCT) {
-        const uint16_t b = f2bf(__ldcg(vr + c));
+        const uint16_t b = f2bf(att_vn[c]);
         M.vc[cofs + c] = b;
         att_vn[c] = bf2f(b);
       }
@@ -567,11 +831,11 @@ __device__ __forceinline__ void attention_phase(const DevModel& M, const StepArg
 #pragma unroll
     for (int e = 0; e < EPL; ++e) {
       acc[j][e] = 0.f;
-      qr[j][e] = (unit && !dry) ? att_q[j * HD + lane * EPL + e] : 0.f;
+      qr[j][e] = att_q[j * HD + lane * EPL + e];
     }
   }
   const float scale = 1.0f / sqrtf(float(HD));
-  MK_CHUNK_LOOP(d, 
+  MK_CHUNK_LOOP(d, {
     const uint16_t* k16 = reinterpret_cast<const uint16_t*>(p0) + lane * EPL;
     const uint16_t* v16 = reinterpret_cast<const uint16_t*>(p1) + lane * EPL;
     float kf[EPL], vf[EPL];
@@ -581,9 +845,9 @@ __device__ __forceinline__ void attention_phase(const DevModel& M, const StepArg
       vf[e] = bf2f(v16[e]);
     }
     att_consume<G, EPL>(am, al, acc, qr, kf, vf, scale);
-  );
-  const bool dry_post = named_sync_or(1, NCT, aborted(t));
-  if (!unit || dry_post) return;
+  });
+  const bool dry_post = named_sync_or(1, NCT, aborted(t) || !work);
+  if (dry_post) return;
   // the new position (not in the cache at launch) goes to the next warp in turn
   if (last && warp == (d.n % NCW)) {
     float kf[EPL], vf[EPL];
@@ -620,8 +884,10 @@ __device__ __forceinline__ void attention_phase(const DevModel& M, const StepArg
     }
     named_sync(1, NCT);
   }
-  float* pbase = M.part + (size_t(gidx) * kMaxCtas + d.unit_s) * G * (HD + 2);
-  for (int i = tid; i < G * HD; i += NCT) pbase[(i / HD) * (HD + 2) + (i % HD)] = att_acc[i];
+  // publish this split's partial as tagged words: per head [acc(HD) | m | l]
+  unsigned long long* part = M.part_ll + size_t(gidx) * kMaxCtas * G * (HD + 2);
+  unsigned long long* pbase = part + size_t(d.unit_s) * G * (HD + 2);
+  for (int i = tid; i < G * HD; i += NCT) ll_put(pbase + (i / HD) * (HD + 2) + (i % HD), att_acc[i], tag_out);
   if (tid < G) {
     float mx = -INFINITY, ls = 0.f;
     for (int w = 0; w < NCW; ++w) mx = fmaxf(mx, att_ml[(w * G + tid) * 2]);
@@ -629,51 +895,147 @@ __device__ __forceinline__ void attention_phase(const DevModel& M, const StepArg
       const float lw = att_ml[(w * G + tid) * 2 + 1];
       if (lw > 0.f) ls += lw * expf(att_ml[(w * G + tid) * 2] - mx);
     }
-    pbase[tid * (HD + 2) + HD] = mx;
-    pbase[tid * (HD + 2) + HD + 1] = ls;
+    ll_put(pbase + tid * (HD + 2) + HD, mx, tag_out);
+    ll_put(pbase + tid * (HD + 2) + HD + 1, ls, tag_out);
   }
-  __threadfence();
-  named_sync(1, NCT);
-  if (tid == 0) {
-    unsigned* tk = M.tickets + L.sub * M.nkv + gidx;
-    const unsigned prev = atomicAdd(tk, 1u);
-    t->flag = (prev == unsigned(d.S - 1)) ? 1 : 0;
-    if (t->flag) atomicExch(tk, 0u);
-  }
-  named_sync(1, NCT);
-  if (t->flag) {
-    // last split of this KV group: merge the S partials into atto
-    __threadfence();
-    for (int i = tid; i < G * HD; i += NCT) {
-      const int j = i / HD, e = i % HD;
-      float mx = -INFINITY;
-      for (int s = 0; s < d.S; ++s)
-        mx = fmaxf(mx, __ldcg(M.part + (size_t(gidx) * kMaxCtas + s) * G * (HD + 2) +
-                              j * (HD + 2) + HD));
-      float num = 0.f, den = 0.f;
-      for (int s = 0; s < d.S; ++s) {
-        const float* pb = M.part + (size_t(gidx) * kMaxCtas + s) * G * (HD + 2) + j * (HD + 2);
-        const float f = expf(__ldcg(pb + HD) - mx);
-        num = fmaf(f, __ldcg(pb + e), num);
-        den = fmaf(f, __ldcg(pb + HD + 1), den);
+  // Cooperative merge: every split CTA of the group merges its slice
+  // [e0, e1) of the group's G*HD outputs from all S partials.  The (m, l)
+  // words of all splits double as the group's completion signal.
+  const int S = d.S;
+  const int e0 = (G * HD) * d.unit_s / S, e1 = (G * HD) * (d.unit_s + 1) / S;
+  const int ne = e1 - e0;
+  constexpr int ATT_SCRATCH = 2 * G * HD + 2 * HD + NCW * G * 2;
+  float* mls = uni + ATT_SCRATCH;  // [S][G][2]  (m, l) of every split
+  float* wgt = mls + S * G * 2;    // [S][G]     merge weights
+  float* stage = uni;              // [S][ne]    the slice's partial values (att_q is free now)
+  bool ok2 = true;
+  {
+    uint64_t start = 0;
+    for (int it = 0;; ++it) {
+      bool stale = false;
+#pragma unroll 4
+      for (int w = tid; w < S * G * 2; w += NCT) {
+        const int si = w / (G * 2), j = (w >> 1) % G, c = w & 1;
+        const unsigned long long v = ll_get(part + (size_t(si) * G + j) * (HD + 2) + HD + c);
+        if (uint32_t(v >> 32) != tag_out) stale = true;
+        else mls[w] = __uint_as_float(uint32_t(v));
       }
-      M.atto[(gidx * G + j) * HD + e] = num / den;
+      if (!stale) break;
+      if (it == 0) start = global_ns();
+      else if ((it & 7) == 0 && give_up(t, M.err, start, a.wait_ns)) { ok2 = false; break; }
     }
   }
+  if (named_sync_or(1, NCT, !ok2)) return;
+  if (tid < G) {
+    float mx = -INFINITY;
+    for (int si = 0; si < S; ++si) mx = fmaxf(mx, mls[(si * G + tid) * 2]);
+    float den = 0.f;
+    for (int si = 0; si < S; ++si) {
+      const float f = expf(mls[(si * G + tid) * 2] - mx);
+      wgt[si * G + tid] = f;
+      den = fmaf(f, mls[(si * G + tid) * 2 + 1], den);
+    }
+    const float inv = 1.0f / den;
+    for (int si = 0; si < S; ++si) wgt[si * G + tid] *= inv;
+  }
+  {
+    uint64_t start = 0;
+    for (int it = 0;; ++it) {
+      bool stale = false;
+#pragma unroll 4
+      for (int w = tid; w < S * ne; w += NCT) {
+        const int si = w / ne, e = e0 + w % ne;
+        const unsigned long long v = ll_get(part + (size_t(si) * G + e / HD) * (HD + 2) + e % HD);
+        if (uint32_t(v >> 32) != tag_out) stale = true;
+        else stage[w] = __uint_as_float(uint32_t(v));
+      }
+      if (!stale) break;
+      if (it == 0) start = global_ns();
+      else if ((it & 7) == 0 && give_up(t, M.err, start, a.wait_ns)) { ok2 = false; break; }
+    }
+  }
+  if (named_sync_or(1, NCT, !ok2)) return;
+  for (int w = tid; w < ne; w += NCT) {
+    const int e = e0 + w, j = e / HD;
+    float o = 0.f;
+    for (int si = 0; si < S; ++si) o = fmaf(wgt[si * G + j], stage[si * ne + w], o);
+    ll_put(M.atto_ll + size_t(gidx) * G * HD + e, o, tag_out);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Cursor over one CTA's chunk schedule for one launch: every phase of every
+// layer, then the LM head, each split into chunks of at most `rpc` rows.
+// ----------------------------------------------------------------------------
+constexpr size_t PF_AHEAD = size_t(256) << 10;  // L2 prefetch distance per CTA (bytes)
+
+struct ChunkCursor {
+  int l, p, np, gp;
+  int kinds[8];
+  PD d;
+  int r;      // first row of the current chunk
+  bool done;
+  __device__ __forceinline__ int nrows() const { return min(d.rpc, d.r0 + d.n - r); }
+  __device__ __forceinline__ uint32_t bytes() const { return uint32_t(nrows()) * d.row_bytes; }
+  __device__ __forceinline__ const char* src0() const { return d.p0 + size_t(r) * d.row_bytes; }
+  __device__ __forceinline__ const char* src1() const { return d.p1 + size_t(r) * d.row_bytes; }
+};
+
+// Move to the first chunk at or after phase (l, p); skips empty phases.
+__device__ __forceinline__ void cursor_settle(ChunkCursor& c, const DevModel& M,
+                                              const StepArgs& a, int cta, uint64_t pol_w,
+                                              uint64_t pol_s) {
+  while (true) {
+    if (c.l > M.n_layers) {
+      c.done = true;
+      return;
+    }
+    if (c.p >= c.np) {
+      ++c.l;
+      c.p = 0;
+      if (c.l < M.n_layers) c.np = layer_phases(M.layers[c.l], c.kinds);
+      else if (c.l == M.n_layers) { c.kinds[0] = PH_LM; c.np = 1; }
+      continue;
+    }
+    c.d = describe(M, a, c.kinds[c.p], c.l < M.n_layers ? c.l : 0, c.gp, cta, pol_w, pol_s);
+    c.r = c.d.r0;
+    if (c.d.n > 0) return;
+    ++c.p;
+    ++c.gp;
+  }
+}
+
+__device__ __forceinline__ void cursor_init(ChunkCursor& c, const DevModel& M, const StepArgs& a,
+                                            int cta, uint64_t pol_w, uint64_t pol_s) {
+  c.l = 0;
+  c.p = 0;
+  c.gp = 0;
+  c.done = false;
+  c.np = layer_phases(M.layers[0], c.kinds);
+  cursor_settle(c, M, a, cta, pol_w, pol_s);
+}
+
+__device__ __forceinline__ void cursor_next(ChunkCursor& c, const DevModel& M, const StepArgs& a,
+                                            int cta, uint64_t pol_w, uint64_t pol_s) {
+  c.r += c.d.rpc;
+  if (c.r < c.d.r0 + c.d.n) return;
+  ++c.p;
+  ++c.gp;
+  cursor_settle(c, M, a, cta, pol_w, pol_s);
 }
 
 // ----------------------------------------------------------------------------
 // the kernel
 // ----------------------------------------------------------------------------
 template <int DK, int HD, int GQ>
-__global__ void __launch_bounds__(NTHR, 1) decode_kernel(const StepArgs a) {
-  using C = Cfg<DK, HD, GQ>;
+__global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__ StepArgs a) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* ring = smem_raw;
   SmemTail* t = reinterpret_cast<SmemTail*>(smem_raw + size_t(NSLOT) * SLOT);
   float* uni = reinterpret_cast<float*>(smem_raw + size_t(NSLOT) * SLOT + sizeof(SmemTail));
+  float* xraw = uni + UNION_FLOATS;
 
-  const DevModel& M = *a.m;
+  const DevModel& M = a.m;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x;
 
@@ -688,7 +1050,6 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const StepArgs a) {
     if (a.tok_src) tok = int(0xFFFFFFFFu - uint32_t(__ldcg(&M.amax[a.amax_in]) & 0xFFFFFFFFull));
     if (tok < 0 || tok >= M.V) tok = 0;
     t->token = tok;
-    if (cta == 0) M.amax[a.amax_out] = 0ull;  // reset before any CTA's atomicMax
     fence_barrier_init();
   }
   // RoPE table for this position (angles in double: pos * theta^(-2i/hd)).
@@ -705,36 +1066,44 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const StepArgs a) {
   const uint64_t pol_s = policy_evict_last();
 
   // ======================= producer warp ====================================
+  // Two cursors walk the same chunk schedule: the load cursor fills the
+  // shared-memory ring (TMA bulk copies, waits for free slots); the prefetch
+  // cursor runs up to PF_AHEAD bytes ahead issuing L2 bulk prefetches, so HBM
+  // keeps streaming while the consumers wait for other CTAs and the ring
+  // refills from L2.
   if (warp == NCW) {
     if (lane != 0) return;
+    ChunkCursor ld, pf;
+    cursor_init(ld, M, a, cta, pol_w, pol_s);
+    cursor_init(pf, M, a, cta, pol_w, pol_s);
+    size_t ld_bytes = 0, pf_bytes = 0;
     uint32_t g = 0;
-    int gp = 0;
-    int kinds[8];
-    for (int l = 0; l <= M.n_layers && !aborted(t); ++l) {
-      int np;
-      if (l < M.n_layers) np = layer_phases(M.layers[l], kinds);
-      else { kinds[0] = PH_LM; np = 1; }
-      for (int p = 0; p < np && !aborted(t); ++p, ++gp) {
-        PD d = describe(M, a, kinds[p], l < M.n_layers ? l : 0, gp, cta, pol_w, pol_s);
-        for (int r = d.r0; r < d.r0 + d.n; r += d.rpc, ++g) {
-          int slot = int(g % NSLOT);
-          if (g >= NSLOT && !bounded_wait(&t->empty[slot], ((g / NSLOT) - 1) & 1, t, M, a.wait_ns))
-            break;
-          int nr = min(d.rpc, d.r0 + d.n - r);
-          uint32_t bytes = uint32_t(nr) * d.row_bytes;
-          unsigned char* dst = ring + size_t(slot) * SLOT;
-          mbar_arrive_expect_tx(&t->full[slot], bytes * (d.p1 ? 2u : 1u));
-          bulk_g2s(dst, d.p0 + size_t(r) * d.row_bytes, bytes, &t->full[slot], d.pol);
-          if (d.p1)
-            bulk_g2s(dst + size_t(d.rpc) * d.row_bytes, d.p1 + size_t(r) * d.row_bytes, bytes,
-                     &t->full[slot], d.pol);
-        }
+    while (!ld.done && !aborted(t)) {
+      // keep the prefetch cursor PF_AHEAD bytes ahead of the loads
+      while (!pf.done && pf_bytes < ld_bytes + PF_AHEAD) {
+        const uint32_t b = pf.bytes();
+        bulk_prefetch_l2(pf.src0(), b);
+        if (pf.d.p1) bulk_prefetch_l2(pf.src1(), b);
+        pf_bytes += size_t(b) * (pf.d.p1 ? 2 : 1);
+        cursor_next(pf, M, a, cta, pol_w, pol_s);
       }
+      const int slot = int(g % NSLOT);
+      if (g >= NSLOT && !bounded_wait(&t->empty[slot], ((g / NSLOT) - 1) & 1, t, M.err, a.wait_ns))
+        break;
+      const uint32_t bytes = ld.bytes();
+      unsigned char* dst = ring + size_t(slot) * SLOT;
+      mbar_arrive_expect_tx(&t->full[slot], bytes * (ld.d.p1 ? 2u : 1u));
+      bulk_g2s(dst, ld.src0(), bytes, &t->full[slot], ld.d.pol);
+      if (ld.d.p1)
+        bulk_g2s(dst + size_t(ld.d.rpc) * ld.d.row_bytes, ld.src1(), bytes, &t->full[slot], ld.d.pol);
+      ld_bytes += size_t(bytes) * (ld.d.p1 ? 2 : 1);
+      ++g;
+      cursor_next(ld, M, a, cta, pol_w, pol_s);
     }
     // Let every copy still in flight land before the CTA may exit.
-    uint32_t first = g > uint32_t(NSLOT) ? g - NSLOT : 0u;
+    const uint32_t first = g > uint32_t(NSLOT) ? g - NSLOT : 0u;
     for (uint32_t q = first; q < g; ++q) {
-      uint64_t start = global_ns();
+      const uint64_t start = global_ns();
       while (!mbar_try_wait(&t->full[q % NSLOT], (q / NSLOT) & 1)) {
         if (global_ns() - start > uint64_t(a.wait_ns)) break;
       }
@@ -746,11 +1115,12 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const StepArgs a) {
   const int tok = t->token;
   const uint16_t* emb_row = M.embed + size_t(tok) * M.H;
   uint32_t g = 0;  // chunk counter (same order as the producer)
-  int gp = 0, nbar = 0;
-  float best_v = -INFINITY;
-  int best_i = 0x7FFFFFFF;
+  int gp = 0;
   int kinds[8];
-  bool first_residual = true;
+  // tags of the latest producer of each tagged buffer
+  uint32_t tag_x = 0, tag_inp = 0, tag_dno = 0, tag_q = 0, tag_k = 0, tag_v = 0, tag_att = 0,
+           tag_h = 0;
+  int xb = 0;  // residual buffer holding the latest x
 
   for (int l = 0; l <= M.n_layers; ++l) {
     const bool lm = (l == M.n_layers);
@@ -762,138 +1132,180 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const StepArgs a) {
     for (int p = 0; p < np; ++p, ++gp) {
       const int kind = kinds[p];
       const PD d = describe(M, a, kind, lm ? 0 : l, gp, cta, pol_w, pol_s);
+      const uint32_t tag_me = make_tag(a.seq, gp);
+      // debug hook: the inputs of phase `fail_phase` carry a tag nobody writes
+      const uint32_t dbg = gp == a.fail_phase ? 0x80000000u : 0u;
       // uniform across the consumer warps (also orders the previous phase)
       const bool dry = named_sync_or(1, NCT, aborted(t));
-      const int row_vecs = int(d.row_bytes / 16);
+      GemvJob j{};  // matrix phases fill it in; one dispatch after the switch
+      j.d = d;
+      j.tag = tag_me;
+      bool gemv = false;
       switch (kind) {
-        case PH_DN_IN: {
-          if (!dry) build_rmsnorm(uni, M.x, l == 0 ? emb_row : nullptr, L.attn_norm, M.H, M.eps, t, tid);
-          float xr[XREG_VEC][8];
-          load_xregs(xr, uni, row_vecs, lane);
-          const float4* conv_st = reinterpret_cast<const float4*>(M.conv_state[a.st_buf]);
-          float4* conv_wr = reinterpret_cast<float4*>(M.conv_state[a.st_buf]);
-          MK_CHUNK_LOOP(d, 
-            float y = warp_sum(row_dot_regs(reinterpret_cast<const uint4*>(p0), xr, row_vecs, lane));
-            if (lane == 0) {
-              if (row < M.ch) {
-                // causal conv (taps u_{t-3}, u_{t-2}, u_{t-1}, u_t) + SiLU, shift the history
-                const size_t ci = size_t(L.sub) * M.ch + row;
-                float4 s = conv_st[ci];
-                uint2 wc = *reinterpret_cast<const uint2*>(L.conv_w + size_t(row) * 4);
-                float c = bf_lo(wc.x) * s.x + bf_hi(wc.x) * s.y + bf_lo(wc.y) * s.z + bf_hi(wc.y) * y;
-                conv_wr[ci] = make_float4(s.y, s.z, y, 0.f);
-                M.inp[row] = siluf_(c);
-              } else {
-                M.inp[row] = y;
+        case PH_DN_IN:
+        case PH_Q:
+        case PH_GU:
+        case PH_LM: {
+          // input: RMSNorm of the residual stream (the embedding at layer 0)
+          bool ok = true;
+          // union layout in this phase: x [0, 2048) | conv history [2048, 3072)
+          // (<= CONV_ROWS_MAX float4) | conv taps [3072, 3584) (<= CONV_ROWS_MAX uint2)
+          float4* conv_s = reinterpret_cast<float4*>(uni + 2048);
+          uint2* conv_taps = reinterpret_cast<uint2*>(uni + 2048 + 4 * CONV_ROWS_MAX);
+          float4* conv_g = reinterpret_cast<float4*>(M.conv_state[a.st_buf]) + size_t(L.sub) * M.ch;
+          if (!dry) {
+            if (kind == PH_DN_IN) {
+              // stage the conv history and taps of this CTA's q|k|v rows first
+              // (independent of the input: their latency overlaps the wait)
+              const int nconv = max(0, min(d.r0 + d.n, M.ch) - d.r0);
+              for (int i = tid; i < nconv; i += NCT) {
+                conv_s[i] = conv_g[d.r0 + i];
+                conv_taps[i] = *reinterpret_cast<const uint2*>(L.conv_w + size_t(d.r0 + i) * 4);
               }
             }
-          );
+            if (l == 0 && kind != PH_GU) {
+              for (int i = tid; i < M.H; i += NCT) uni[i] = bf2f(emb_row[i]);
+            } else {
+              ok = ll_gather<per_thread(XRAW_MAX)>(uni, M.x_ll + size_t(xb) * M.H, M.H,
+                                                   tag_x | dbg, t, M.err, a.wait_ns, tid);
+            }
+          }
+          const bool bad = named_sync_or(1, NCT, !ok);
+          if (!dry && !bad) {
+            const uint16_t* gain = kind == PH_GU ? L.mlp_norm
+                                   : kind == PH_LM ? M.final_norm : L.attn_norm;
+            rmsnorm_inplace(uni, kind == PH_LM ? nullptr : xraw, gain, M.H, M.eps, t, tid);
+          }
+          gemv = true;
+          j.shape = gemv_shape(M.H);
+          if (kind == PH_DN_IN) {
+            j.epi = EPI_INPROJ;
+            j.dst = M.inp_ll;
+            j.conv_s = conv_s;
+            j.conv_taps = conv_taps;
+            j.conv_out = conv_g;
+            j.ch = M.ch;
+            tag_inp = tag_me;
+          } else if (kind == PH_Q) {
+            j.epi = EPI_STORE;
+            j.dst = M.qkv_ll;
+            tag_q = tag_me;
+          } else if (kind == PH_GU) {
+            j.epi = EPI_SWIGLU;
+            j.dst = M.mlph_ll;
+            tag_h = tag_me;
+          } else {
+            j.epi = EPI_LOGITS;
+            j.logits = a.logits;
+          }
           break;
         }
-        case PH_Q:
         case PH_K:
         case PH_V: {
-          if (kind == PH_Q && !dry)
-            build_rmsnorm(uni, M.x, l == 0 ? emb_row : nullptr, L.attn_norm, M.H, M.eps, t, tid);
-          float xr[XREG_VEC][8];
-          load_xregs(xr, uni, row_vecs, lane);
-          const int off = kind == PH_Q ? 0 : (kind == PH_K ? M.nq * HD : (M.nq + M.nkv) * HD);
-          MK_CHUNK_LOOP(d, 
-            float y = warp_sum(row_dot_regs(reinterpret_cast<const uint4*>(p0), xr, row_vecs, lane));
-            if (lane == 0) M.qkv[off + row] = y;
-          );
+          gemv = true;
+          j.shape = gemv_shape(M.H);
+          j.epi = EPI_STORE;
+          j.dst = M.qkv_ll + (kind == PH_K ? M.nq * HD : (M.nq + M.nkv) * HD);
+          if (kind == PH_K) tag_k = tag_me;
+          else tag_v = tag_me;
           break;
         }
-        case PH_GU: {
-          if (!dry) build_rmsnorm(uni, M.x, nullptr, L.mlp_norm, M.H, M.eps, t, tid);
-          float xr[XREG_VEC][8];
-          load_xregs(xr, uni, row_vecs, lane);
-          MK_CHUNK_LOOP(d, 
-            float yg = warp_sum(row_dot_regs(reinterpret_cast<const uint4*>(p0), xr, row_vecs, lane));
-            float yu = warp_sum(row_dot_regs(reinterpret_cast<const uint4*>(p1), xr, row_vecs, lane));
-            if (lane == 0) M.mlph[row] = siluf_(yg) * yu;
-          );
-          break;
-        }
-        case PH_OUT:
-        case PH_DOWN: {
+        case PH_OUT: {
+          bool ok = true;
+          const int K = L.is_attn ? M.nq * M.hd : M.nh * M.dv;
           if (!dry) {
-            if (kind == PH_DOWN) build_copy(uni, M.mlph, M.I, tid);
-            else if (L.is_attn) build_copy(uni, M.atto, M.nq * M.hd, tid);
-            else build_gated_norm<DK>(uni, M, L, tid);
+            if (L.is_attn) {
+              ok = ll_gather<per_thread(UNION_FLOATS)>(uni, M.atto_ll, K, tag_att | dbg, t, M.err,
+                                                       a.wait_ns, tid);
+            } else {
+              // gated RMSNorm of the readout: o_h from the state phase, z_h
+              // from the in-projection (z staged in the upper half of uni)
+              // o (tagged by the state phase) and z (by the in-projection)
+              // in one polling round
+              const LLSeg sg[2] = {{M.dno_ll, uni, K, tag_dno | dbg},
+                                   {M.inp_ll + M.ch, uni + 2048, K, tag_inp}};
+              ok = ll_gather_segs<per_thread(4096), 2>(sg, t, M.err, a.wait_ns, tid);
+            }
           }
-          const bool first = kind == PH_OUT && first_residual;
-          float* hid = kind == PH_DOWN ? a.hidden : nullptr;
-          if (row_vecs <= XREG_VEC * 32) {
-            float xr[XREG_VEC][8];
-            load_xregs(xr, uni, row_vecs, lane);
-            MK_CHUNK_LOOP(d, 
-              float y = warp_sum(row_dot_regs(reinterpret_cast<const uint4*>(p0), xr, row_vecs, lane));
-              if (lane == 0) {
-                float xn = (first ? bf2f(emb_row[row]) : __ldcg(M.x + row)) + y;
-                M.x[row] = xn;
-                if (hid) hid[size_t(l) * M.H + row] = xn;
+          const bool bad = named_sync_or(1, NCT, !ok);
+          if (!dry && !bad && !L.is_attn) {
+            constexpr int EPL = DK / 32;  // dv == dk
+            for (int h = warp; h < M.nh; h += NCW) {
+              float o[EPL];
+              float ss = 0.f;
+#pragma unroll
+              for (int e = 0; e < EPL; ++e) {
+                o[e] = uni[h * DK + lane * EPL + e];
+                ss = fmaf(o[e], o[e], ss);
               }
-            );
-          } else {
-            MK_CHUNK_LOOP(d, 
-              float y = warp_sum(row_dot_smem(reinterpret_cast<const uint4*>(p0), uni, row_vecs, lane));
-              if (lane == 0) {
-                float xn = (first ? bf2f(emb_row[row]) : __ldcg(M.x + row)) + y;
-                M.x[row] = xn;
-                if (hid) hid[size_t(l) * M.H + row] = xn;
+              ss = warp_sum(ss);
+              const float inv = 1.0f / sqrtf(ss / float(DK) + M.eps);
+#pragma unroll
+              for (int e = 0; e < EPL; ++e) {
+                const int i = lane * EPL + e;
+                uni[h * DK + i] =
+                    o[e] * inv * bf2f(L.out_norm[i]) * siluf_(uni[2048 + h * DK + i]);
               }
-            );
+            }
+            named_sync(1, NCT);
           }
-          if (kind == PH_OUT) first_residual = false;
+          gemv = true;
+          j.shape = gemv_shape(K);
+          j.epi = EPI_RESID;
+          j.dst = M.x_ll + size_t(xb ^ 1) * M.H;
+          j.xraw = xraw;
+          xb ^= 1;
+          tag_x = tag_me;
           break;
         }
-        case PH_LM: {
-          if (!dry) build_rmsnorm(uni, M.x, nullptr, M.final_norm, M.H, M.eps, t, tid);
-          float xr[XREG_VEC][8];
-          load_xregs(xr, uni, row_vecs, lane);
-          float* logits = a.logits;
-          MK_CHUNK_LOOP(d, 
-            float y = warp_sum(row_dot_regs(reinterpret_cast<const uint4*>(p0), xr, row_vecs, lane));
-            if (lane == 0) {
-              logits[row] = y;
-              if (y > best_v || (y == best_v && row < best_i)) { best_v = y; best_i = row; }
-            }
-          );
+        case PH_DOWN: {
+          bool ok = true;
+          if (!dry)
+            ok = ll_gather<per_thread(UNION_FLOATS)>(uni, M.mlph_ll, M.I, tag_h | dbg, t, M.err,
+                                                     a.wait_ns, tid);
+          named_sync_or(1, NCT, !ok);
+          gemv = true;
+          j.shape = gemv_shape(M.I);
+          j.epi = EPI_RESID;
+          j.dst = M.x_ll + size_t(xb ^ 1) * M.H;
+          j.xraw = xraw;
+          j.hidden = a.hidden ? a.hidden + size_t(l) * M.H : nullptr;
+          xb ^= 1;
+          tag_x = tag_me;
           break;
         }
         case PH_DN_ST:
-          dn_state_phase<DK>(M, a, L, d, g, ring, t, uni, dry, tid, warp, lane);
+          dn_state_phase<DK>(M, a, L, d, g, ring, t, uni, tag_inp | dbg, tag_me, dry, tid, warp,
+                             lane);
+          tag_dno = tag_me;
           break;
         case PH_ATT:
-          attention_phase<HD, GQ>(M, a, L, d, g, ring, t, uni, dry, tid, warp, lane);
+          attention_phase<HD, GQ>(M, a, L, d, g, ring, t, uni, tag_q | dbg, tag_k, tag_v, tag_me,
+                                  dry, tid, warp, lane);
+          tag_att = tag_me;
           break;
         default:
           break;
       }
-
-      if (has_grid_barrier(kind)) {
-        named_sync(1, NCT);
-        if (tid == 0) grid_barrier(M, a, nbar, t);
-        ++nbar;
-        named_sync(1, NCT);
-      }
+      if (gemv) g = gemv_dispatch(j, g, ring, t, M.err, a.wait_ns, uni);
     }
   }
 
   // ---------------- argmax over the grid ----------------
-  if (lane == 0 && best_i != 0x7FFFFFFF) atomicMax(&t->best, pack_argmax(best_v, best_i));
-  named_sync(1, NCT);
-  if (tid == 0 && !aborted(t)) {
+  const bool bad = named_sync_or(1, NCT, aborted(t));
+  if (tid == 0 && !bad) {
     if (t->best) atomicMax(&M.amax[a.amax_out], t->best);
     __threadfence();
-    unsigned* tk = M.tickets + M.n_attn * M.nkv;
-    unsigned prev = atomicAdd(tk, 1u);
+    unsigned* tk = M.tickets;
+    const unsigned prev = atomicAdd(tk, 1u);
     if (prev == unsigned(M.ncta - 1)) {
       atomicExch(tk, 0u);
       __threadfence();
-      unsigned long long v = atomicAdd(&M.amax[a.amax_out], 0ull);
+      const unsigned long long v = atomicAdd(&M.amax[a.amax_out], 0ull);
       if (a.tok_out) *a.tok_out = int(0xFFFFFFFFu - uint32_t(v & 0xFFFFFFFFull));
+      // every CTA has read its input token by now: clear the slot the next
+      // launch accumulates into
+      M.amax[a.amax_in] = 0ull;
     }
   }
 }

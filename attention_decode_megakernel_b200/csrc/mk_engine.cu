@@ -22,7 +22,7 @@ struct Layout {
   size_t model;
   size_t dn_state[mk::kStateBufs], conv_state[mk::kStateBufs];
   size_t kc, vc;
-  size_t x, inp, dno, qkv, atto, mlph, part, hidden, logits, tickets, bar, err, amax;
+  size_t x, inp, dno, qkv, atto, mlph, part, hidden, logits, tickets, err, amax;
   size_t total;
 };
 
@@ -64,17 +64,16 @@ Layout make_layout(const mk_config& c) {
   const size_t kv = size_t(n_attn) * c.kv_heads * c.max_ctx * c.head_dim * 2;
   L.kc = take(kv);
   L.vc = take(kv);
-  L.x = take(M * c.hidden * 4);
-  L.inp = take(M * rin * 4);
-  L.dno = take(M * c.dn_heads * c.dn_dv * 4);
-  L.qkv = take(M * size_t(c.q_heads + 2 * c.kv_heads) * c.head_dim * 4);
-  L.atto = take(M * size_t(c.q_heads) * c.head_dim * 4);
-  L.mlph = take(M * size_t(c.mlp) * 4);
-  L.part = take(size_t(c.kv_heads) * mk::kMaxCtas * M * G * (c.head_dim + 2) * 4);
+  L.x = take(2 * M * c.hidden * 8);
+  L.inp = take(M * rin * 8);
+  L.dno = take(M * c.dn_heads * c.dn_dv * 8);
+  L.qkv = take(M * size_t(c.q_heads + 2 * c.kv_heads) * c.head_dim * 8);
+  L.atto = take(M * size_t(c.q_heads) * c.head_dim * 8);
+  L.mlph = take(M * size_t(c.mlp) * 8);
+  L.part = take(size_t(c.kv_heads) * mk::kMaxCtas * M * G * (c.head_dim + 2) * 8);
   L.hidden = take(size_t(c.n_layers) * c.hidden * 4);
   L.logits = take(size_t(c.vocab) * 4);
-  L.tickets = take((size_t(n_attn) * c.kv_heads + 1) * 4);
-  L.bar = take(4);
+  L.tickets = take(4);
   L.err = take(4);
   L.amax = take(2 * 8);
   L.total = off;
@@ -118,14 +117,13 @@ struct mk_engine {
   int ncta;
   int pos;
   int cur_buf;
-  unsigned bar_epoch;
+  uint32_t seq;  // launch sequence number for activation tags
   int amax_toggle;
   int pending_verify;
   int verify_bufs[mk::kMaxVerify];
   int64_t launches;
   long long wait_ns;
-  int fail_barrier;
-  int nbar_decode;
+  int fail_phase;
 };
 
 namespace {
@@ -150,7 +148,7 @@ int read_device_error(mk_engine* e) {
 int launch_decode(mk_engine* e, int pos, int st_buf, int token, int tok_src, float* logits,
                   int32_t* tok_out) {
   mk::StepArgs a;
-  a.m = e->dm;
+  a.m = e->hm;
   a.pos = pos;
   a.token = token;
   a.tok_src = tok_src;
@@ -160,10 +158,11 @@ int launch_decode(mk_engine* e, int pos, int st_buf, int token, int tok_src, flo
   a.logits = logits ? logits : reinterpret_cast<float*>(e->ws + e->lay.logits);
   a.tok_out = tok_out;
   a.hidden = reinterpret_cast<float*>(e->ws + e->lay.hidden);
-  a.bar_base = e->bar_epoch;
-  a.fail_barrier = e->fail_barrier;
+  e->seq = e->seq + 1 >= (1u << 23) ? 1u : e->seq + 1;
+  a.seq = e->seq;
+  a.fail_phase = e->fail_phase;
   a.wait_ns = e->wait_ns;
-  e->fail_barrier = -1;
+  e->fail_phase = -1;
   void* args[] = {&a};
   cudaError_t err = cudaLaunchCooperativeKernel(e->var->fn, dim3(e->ncta), dim3(mk::NTHR), args,
                                                 e->var->smem, e->stream);
@@ -171,7 +170,6 @@ int launch_decode(mk_engine* e, int pos, int st_buf, int token, int tok_src, flo
     cudaGetLastError();
     return MK_ERR_LAUNCH;
   }
-  e->bar_epoch += unsigned(e->nbar_decode) * unsigned(e->ncta);
   e->amax_toggle ^= 1;
   e->launches += 1;
   return MK_OK;
@@ -204,6 +202,7 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
   if (c.hidden % 256 || c.hidden > 2048 || c.mlp % 8 || c.mlp > 4096) return MK_ERR_UNSUPPORTED;
   if (c.dn_heads * c.dn_dv > 4096 || c.q_heads * c.head_dim > 4096) return MK_ERR_UNSUPPORTED;
   if (2 * c.mlp > mk::SLOT || c.head_dim * 2 * 2 > mk::SLOT) return MK_ERR_UNSUPPORTED;
+  if (c.dn_heads * c.dn_dv > 2048 || c.mlp > mk::UNION_FLOATS) return MK_ERR_UNSUPPORTED;
 
   // weights: present and 16-byte aligned
   if (!aligned16(w->embed) || !aligned16(w->final_norm)) return MK_ERR_ARG;
@@ -230,6 +229,13 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
   cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
   if (!coop || nsm <= 0) return MK_ERR_LAUNCH;
   const int ncta = nsm < mk::kMaxCtas ? nsm : mk::kMaxCtas;
+  {
+    // attention merge scratch: (m, l) and weights of every split
+    const int smax = ncta / c.kv_heads;
+    const int att = 2 * G * c.head_dim + 2 * c.head_dim + mk::NCW * G * 2;
+    if (att + smax * G * 3 > mk::UNION_FLOATS || G * c.head_dim + smax > att)
+      return MK_ERR_UNSUPPORTED;
+  }
   if (cudaFuncSetAttribute(var->fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            int(var->smem)) != cudaSuccess) {
     cudaGetLastError();
@@ -242,11 +248,15 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
     cudaGetLastError();
     return MK_ERR_LAUNCH;
   }
-  // the DeltaNet head cache must hold every head a CTA's state rows touch
+  // the DeltaNet head cache, row values and conv staging must fit a CTA's
+  // shared scratch
+  if ((2 * c.dn_heads * c.dn_dk + 2 * c.dn_heads * c.dn_dv + 2 * c.dn_heads + ncta - 1) / ncta >
+      mk::CONV_ROWS_MAX)
+    return MK_ERR_UNSUPPORTED;
   {
     int rows = (c.dn_heads * c.dn_dv + ncta - 1) / ncta;
     int heads = rows / c.dn_dv + 2;
-    if (heads * (2 * c.dn_dk + 4) > 4096) return MK_ERR_UNSUPPORTED;
+    if (heads > mk::DN_HEADS_MAX || rows > mk::DN_ROWS_MAX) return MK_ERR_UNSUPPORTED;
   }
 
   mk_engine* e = new (std::nothrow) mk_engine();
@@ -259,8 +269,7 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
   e->var = var;
   e->ncta = ncta;
   e->wait_ns = 2000000000LL;
-  e->fail_barrier = -1;
-  e->nbar_decode = 5 * c.n_layers;
+  e->fail_phase = -1;
 
   DevModel& m = e->hm;
   std::memset(&m, 0, sizeof m);
@@ -315,17 +324,17 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
   }
   m.kc = reinterpret_cast<uint16_t*>(ws + lay.kc);
   m.vc = reinterpret_cast<uint16_t*>(ws + lay.vc);
-  m.x = reinterpret_cast<float*>(ws + lay.x);
-  m.inp = reinterpret_cast<float*>(ws + lay.inp);
-  m.dno = reinterpret_cast<float*>(ws + lay.dno);
-  m.qkv = reinterpret_cast<float*>(ws + lay.qkv);
-  m.atto = reinterpret_cast<float*>(ws + lay.atto);
-  m.mlph = reinterpret_cast<float*>(ws + lay.mlph);
-  m.part = reinterpret_cast<float*>(ws + lay.part);
+  using ull = unsigned long long;
+  m.x_ll = reinterpret_cast<ull*>(ws + lay.x);
+  m.inp_ll = reinterpret_cast<ull*>(ws + lay.inp);
+  m.dno_ll = reinterpret_cast<ull*>(ws + lay.dno);
+  m.qkv_ll = reinterpret_cast<ull*>(ws + lay.qkv);
+  m.atto_ll = reinterpret_cast<ull*>(ws + lay.atto);
+  m.mlph_ll = reinterpret_cast<ull*>(ws + lay.mlph);
+  m.part_ll = reinterpret_cast<ull*>(ws + lay.part);
   m.hidden = reinterpret_cast<float*>(ws + lay.hidden);
   m.logits_scratch = reinterpret_cast<float*>(ws + lay.logits);
   m.tickets = reinterpret_cast<unsigned*>(ws + lay.tickets);
-  m.bar = reinterpret_cast<unsigned*>(ws + lay.bar);
   m.err = reinterpret_cast<int*>(ws + lay.err);
   m.amax = reinterpret_cast<unsigned long long*>(ws + lay.amax);
   e->dm = reinterpret_cast<DevModel*>(ws + lay.model);
@@ -363,7 +372,6 @@ int mk_reset(mk_engine* e) {
   if (r != cudaSuccess) return cuda_status(r);
   e->pos = 0;
   e->cur_buf = 0;
-  e->bar_epoch = 0;
   e->amax_toggle = 0;
   e->pending_verify = 0;
   return MK_OK;
@@ -539,10 +547,10 @@ int mk_get_hidden(mk_engine* e, float* hidden_out) {
 
 int64_t mk_launch_count(const mk_engine* e) { return e ? e->launches : -1; }
 
-int mk_debug_set_wait_limit(mk_engine* e, int64_t limit_ns, int fail_barrier) {
+int mk_debug_set_wait_limit(mk_engine* e, int64_t limit_ns, int fail_phase) {
   if (!e || limit_ns <= 0) return MK_ERR_ARG;
   e->wait_ns = limit_ns;
-  e->fail_barrier = fail_barrier;
+  e->fail_phase = fail_phase;
   return MK_OK;
 }
 

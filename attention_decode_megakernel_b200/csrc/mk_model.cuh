@@ -37,18 +37,18 @@ struct DevModel {
   float *dn_state[kStateBufs];      // [n_dn][nh][dv][dk]
   float *conv_state[kStateBufs];    // [n_dn][ch][4]  (3 taps of history + pad)
   uint16_t *kc, *vc;                // [n_attn][nkv][max_ctx][hd]
-  // activations (M = max_verify rows where noted)
-  float *x;        // [M][H]      residual stream
-  float *inp;      // [M][rin]    in-proj output: conv'd q|k|v, raw z|b|a
-  float *dno;      // [M][nh*dv]  DeltaNet readout o = S q
-  float *qkv;      // [M][(nq+2nkv)*hd] raw attention projections
-  float *atto;     // [M][nq*hd]  attention output (merged)
-  float *mlph;     // [M][I]      SiLU(gate)*up
-  float *part;     // [nkv][kMaxCtas][M*group][hd+2] split-K attention partials
+  // activations exchanged between CTAs, as tagged words {fp32 value, tag}
+  // (M = max_verify rows where noted)
+  unsigned long long *x_ll;     // [2][M][H]  residual stream (double-buffered)
+  unsigned long long *inp_ll;   // [M][rin]   in-proj output: conv'd q|k|v, raw z|b|a
+  unsigned long long *dno_ll;   // [M][nh*dv] DeltaNet readout o = S q
+  unsigned long long *qkv_ll;   // [M][(nq+2nkv)*hd] raw attention projections
+  unsigned long long *atto_ll;  // [M][nq*hd] attention output (merged)
+  unsigned long long *mlph_ll;  // [M][I]     SiLU(gate)*up
+  unsigned long long *part_ll;  // [nkv][kMaxCtas][M*group][hd+2] split-K attention partials (tagged)
   float *hidden;   // [n_layers][H] residual after each layer (last position)
   float *logits_scratch;  // [V]
-  unsigned *tickets;      // [n_attn*nkv + 1] merge / argmax tickets
-  unsigned *bar;          // grid barrier counter
+  unsigned *tickets;      // [1] grid argmax ticket
   int *err;               // first device error code
   unsigned long long *amax;  // [2] packed argmax slots
 };

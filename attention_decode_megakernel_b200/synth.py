@@ -93,6 +93,16 @@ def tiny_config(max_ctx: int = 256) -> ModelConfig:
         rms_eps=1e-6, max_ctx=max_ctx, max_verify=8)
 
 
+def hybrid_mid_config(max_ctx: int = 512) -> ModelConfig:
+    """The 0.8B layer shapes in 4 layers [DN, DN, DN, Attn] with vocab 4096:
+    full-width vectors and multi-chunk phases at a size the oracle runs fast."""
+    return ModelConfig(
+        name="hybrid-mid-4L-h1024", layer_is_attn=(False, False, False, True),
+        hidden=1024, vocab=4096, mlp=3584, dn_heads=16, dn_dk=128, dn_dv=128,
+        conv_k=4, q_heads=8, kv_heads=2, head_dim=256, rope_theta=1e7,
+        rms_eps=1e-6, max_ctx=max_ctx, max_verify=8)
+
+
 def hybrid_08b_config(max_ctx: int = 4096) -> ModelConfig:
     """24 layers (3 DN + 1 Attn) x 6, hidden 1024, vocab 151936, tied."""
     pattern = tuple([False, False, False, True] * 6)

@@ -38,7 +38,41 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--mode", choices=["full", "kernel"], default="full",
+                   help="kernel: W+K single decode launches at context 520 on a "
+                        "seeded synthetic state (small case for profilers)")
     return p.parse_args()
+
+
+def run_kernel_mode(args):
+    """W warm-up + K timed decode launches at context 520 (one engine)."""
+    import numpy as np
+    import torch
+
+    import attention_decode_megakernel_b200 as mk
+    from attention_decode_megakernel_b200 import build, synth
+    build.build()
+    cfg = synth.hybrid_08b_config(max_ctx=PROMPT + 64)
+    w = synth.make_weights(cfg)
+    eng = mk.Engine(cfg, w)
+    st = synth.make_engine_state(cfg, ctx=PROMPT)
+    dev = {k: (torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v).cuda()
+               if isinstance(v, np.ndarray) else v) for k, v in st.items()}
+    eng.set_state(dev)
+    logits = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
+    for _ in range(args.warmup):
+        eng.decode_step(1, logits)
+    eng.sync()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(eng.stream)
+    for _ in range(args.steps):
+        eng.decode_step(1, logits)
+    e1.record(eng.stream)
+    eng.sync()
+    ms = e0.elapsed_time(e1) / max(args.steps, 1)
+    print(json.dumps({"mode": "kernel", "launches": args.warmup + args.steps,
+                      "ms_per_launch": ms,
+                      "GBps": decode_bytes(cfg, PROMPT + args.warmup) / ms / 1e6}), flush=True)
 
 
 def peaks():
@@ -191,6 +225,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.mode == "kernel":
+        run_kernel_mode(args)
         return
 
     import numpy as np

@@ -184,12 +184,14 @@ int mk_get_hidden(mk_engine *e, float *hidden_out);
 /* Launch statistics: number of kernels the engine launched so far. */
 int64_t mk_launch_count(const mk_engine *e);
 
-/* Debug: device-side wait limit in nanoseconds (default 2e9).  A grid
- * barrier, pipeline or peer wait that exceeds it records MK_ERR_TIMEOUT and
- * the kernel returns early.  `fail_barrier` >= 0 makes the next decode
- * launch wait at that barrier for one arrival more than the grid provides,
- * so the wait must run out (tests of the timeout path only). */
-int mk_debug_set_wait_limit(mk_engine *e, int64_t limit_ns, int fail_barrier);
+/* Debug: device-side wait limit in nanoseconds (default 2e9).  A pipeline
+ * wait or a wait for another CTA's data that exceeds it records
+ * MK_ERR_TIMEOUT and the kernel returns early.  `fail_phase` >= 0 makes the
+ * next decode launch wait, in that phase (0-based index of the launch's
+ * phase sequence: five phases per DeltaNet layer, seven per attention
+ * layer), for data tagged with a value no phase ever writes, so the wait
+ * must run out (tests of the timeout path only). */
+int mk_debug_set_wait_limit(mk_engine *e, int64_t limit_ns, int fail_phase);
 
 /* ------------------------------------------------------------------------
  * Isolated gated delta-rule step (no engine).  One launch advances B

@@ -85,6 +85,28 @@ def test_tiny_prompt_then_greedy_teacher_forced(mk):
     print(tr.finish())
 
 
+def test_mid_prompt_then_greedy_teacher_forced(mk):
+    """0.8B layer shapes (4 layers): 100-token prompt (multi-split attention)
+    then 16 greedy steps, every position compared."""
+    cfg = synth.hybrid_mid_config(max_ctx=256)
+    w = synth.make_weights(cfg)
+    eng = mk.Engine(cfg, w)
+    orc = oracle.OracleModel(cfg, w)
+    tr = Tracker()
+    prompt = synth.make_tokens(cfg.vocab, 100)
+    logits = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
+    for t in prompt:
+        eng.decode_step(int(t), logits)
+        ref, ref_h = orc.step(int(t), want_hidden=True)
+        eng.sync()
+        tr.logits(_np(logits), ref)
+        tr.hidden(_np(eng.get_hidden()), ref_h)
+    _check_state(eng, orc)
+    _teacher_forced(eng, orc, cfg, int(np.argmax(ref)), 16, tr)
+    _check_state(eng, orc)
+    print(tr.finish())
+
+
 def test_tiny_prefill_matches_decode_loop(mk):
     cfg = synth.tiny_config(max_ctx=256)
     w = synth.make_weights(cfg)
@@ -206,20 +228,23 @@ def test_engine_errors(mk):
     assert e.value.code == mk.MK_ERR_ARG
 
 
-def test_barrier_wait_limit_reports_timeout_and_recovers(mk):
-    """A barrier whose count can never be reached (one arrival more than the
-    grid has) must give up after the wait limit, report MK_ERR_TIMEOUT and
-    leave the context usable; mk_reset recovers the engine."""
+@pytest.mark.parametrize("phase", [1, 3, 9, 18, 19, 22])
+def test_wait_limit_reports_timeout_and_recovers(mk, phase):
+    """A phase whose inputs wait for a tag nobody writes must give up after the
+    wait limit, report MK_ERR_TIMEOUT and leave the context usable; mk_reset
+    recovers the engine.  Tiny model phases: 1 DeltaNet state update, 3 first
+    MLP gate/up, 9 second layer's down projection, 18 attention (queries),
+    19 attention output projection, 22 LM head."""
     cfg = synth.tiny_config(max_ctx=64)
     w = synth.make_weights(cfg)
     eng = mk.Engine(cfg, w)
-    eng.set_wait_limit(50_000_000, fail_barrier=3)  # 50 ms
+    eng.set_wait_limit(50_000_000, phase)  # 50 ms
     eng.decode_step(3)
     with pytest.raises(mk.MkError) as e:
         eng.sync()
     assert e.value.code == mk.MK_ERR_TIMEOUT
     eng.reset()
-    eng.set_wait_limit(2_000_000_000, -1)
+    eng.set_wait_limit(2_000_000_000, -1)  # default limit, no failing phase
     orc = oracle.OracleModel(cfg, w)
     tr = Tracker()
     _teacher_forced(eng, orc, cfg, 3, 3, tr)
