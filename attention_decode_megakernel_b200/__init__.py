@@ -87,6 +87,7 @@ def lib():
             "mk_debug_set_wait_limit": (C.c_int, [vp, i64, C.c_int]),
             "mk_delta_step": (C.c_int, [vp, vp, vp, vp, vp, vp, vp, C.c_int, C.c_int,
                                         C.c_int, C.c_int, vp]),
+            "mk_debug_gemm": (C.c_int, [vp, vp, vp, C.c_int, C.c_int, C.c_int, vp]),
             "mk_strerror": (C.c_char_p, [C.c_int]),
         }
         for name, (res, args) in sig.items():
@@ -268,3 +269,16 @@ def mk_delta_step(S, q, k, v, alpha, beta, o, stream=None):
     _check(lib().mk_delta_step(_ptr(S), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                                _ptr(o), int(B), int(heads), int(dk), int(dv), st),
            "mk_delta_step")
+
+
+def mk_debug_gemm(W, X, Cout, stream=None):
+    """C = X W^T on the prompt path's tensor-core GEMM (bf16 in, fp32 out)."""
+    n_out, K = W.shape
+    if X.numel() % (2 * K):
+        raise ValueError("X must hold [2][T][K] bf16 (hi then lo operands)")
+    T = X.numel() // (2 * K)
+    if Cout.numel() != T * n_out:
+        raise ValueError("C must hold [T][n_out] float32")
+    st = stream if stream is not None else 0
+    _check(lib().mk_debug_gemm(_ptr(W), _ptr(X), _ptr(Cout), int(n_out), int(T), int(K), st),
+           "mk_debug_gemm")

@@ -11,6 +11,7 @@
 #include "mk_decode.cuh"
 #include "mk_delta.cuh"
 #include "mk_model.cuh"
+#include "mk_prefill.cuh"
 
 namespace {
 
@@ -23,8 +24,14 @@ struct Layout {
   size_t dn_state[mk::kStateBufs], conv_state[mk::kStateBufs];
   size_t kc, vc;
   size_t x, inp, dno, qkv, atto, mlph, part, hidden, logits, tickets, err, amax;
+  // multi-token prompt path: T_MAX positions per chunk
+  int tmax, pw, aw;
+  size_t pf_tok, pf_x, pf_xn, pf_p, pf_o, pf_a16, pf_qk, pf_bak;
   size_t total;
 };
+
+constexpr int kPrefillChunk = 1024;  // most positions one prompt chunk processes
+constexpr int kPrefillMinBatch = 8;  // shorter prompts run as decode steps
 
 int count_attn(const mk_config& c) {
   int n = 0;
@@ -76,8 +83,67 @@ Layout make_layout(const mk_config& c) {
   L.tickets = take(4);
   L.err = take(4);
   L.amax = take(2 * 8);
+  {
+    const int T = c.max_ctx < kPrefillChunk ? c.max_ctx : kPrefillChunk;
+    const int nqkv = (c.q_heads + 2 * c.kv_heads) * c.head_dim;
+    int pw = int(rin);
+    if (2 * c.mlp > pw) pw = 2 * c.mlp;
+    if (nqkv > pw) pw = nqkv;
+    int aw = c.dn_heads * c.dn_dv;
+    if (c.mlp > aw) aw = c.mlp;
+    if (c.q_heads * c.head_dim > aw) aw = c.q_heads * c.head_dim;
+    L.tmax = T;
+    L.pw = pw;
+    L.aw = aw;
+    L.pf_tok = take(size_t(T) * 4);
+    L.pf_x = take(size_t(T) * c.hidden * 4);
+    L.pf_xn = take(size_t(2) * T * c.hidden * 2);  // [hi|lo][T][H] bf16
+    L.pf_p = take(size_t(T) * pw * 4);
+    L.pf_o = take(size_t(T) * c.dn_heads * c.dn_dv * 4);
+    L.pf_a16 = take(size_t(2) * T * aw * 2);  // [hi|lo][T][aw] bf16
+    L.pf_qk = take(size_t(c.dn_heads) * T * 2 * c.dn_dk * 4);
+    L.pf_bak = take(size_t(c.dn_heads) * T * 16);
+  }
   L.total = off;
   return L;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
+// 2D bf16 matrix [rows][cols] (row pitch in elements) as TMA tiles of
+// box_rows x 64 columns with the 128-byte swizzle the MMA descriptors expect.
+bool make_map(CUtensorMap* m, const void* base, int rows, int cols, int pitch, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || (reinterpret_cast<uintptr_t>(base) & 15u) || cols % 64 || (pitch * 2) % 16)
+    return false;
+  const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(pitch) * 2};
+  const cuuint32_t box[2] = {64u, cuuint32_t(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 struct Variant {
@@ -124,6 +190,12 @@ struct mk_engine {
   int64_t launches;
   long long wait_ns;
   int fail_phase;
+  // multi-token prompt path
+  bool pf_ok;
+  struct LayerMaps {
+    CUtensorMap in_proj, out, q, k, v, gate, up, down;
+  } maps[MK_MAX_LAYERS];
+  CUtensorMap map_xn, map_a16_dn, map_a16_mlp, map_a16_att;
 };
 
 namespace {
@@ -172,6 +244,108 @@ int launch_decode(mk_engine* e, int pos, int st_buf, int token, int tok_src, flo
   }
   e->amax_toggle ^= 1;
   e->launches += 1;
+  return MK_OK;
+}
+
+int launch_gemm(mk_engine* e, const CUtensorMap& tw, const CUtensorMap& tx, float* c, int ldc,
+                int n_out, int T, int K, int accumulate) {
+  mk::pf::GemmArgs g;
+  g.tw = tw;
+  g.tx = tx;
+  g.c = c;
+  g.ldc = ldc;
+  g.n_out = n_out;
+  g.T = T;
+  g.K = K;
+  g.accumulate = accumulate;
+  g.x_lo_row = e->lay.tmax;
+  g.err = e->hm.err;
+  g.wait_ns = e->wait_ns;
+  const dim3 grid((n_out + mk::pf::BM - 1) / mk::pf::BM, (T + mk::pf::BN - 1) / mk::pf::BN);
+  mk::pf::gemm_tc<<<grid, mk::pf::GEMM_THREADS, mk::pf::GEMM_SMEM, e->stream>>>(g);
+  e->launches += 1;
+  return cuda_status(cudaGetLastError());
+}
+
+// The stack over T prompt positions starting at e->pos (no logits).
+int prefill_chunk(mk_engine* e, const int32_t* tokens_host, int T) {
+  using namespace mk::pf;
+  const mk_config& c = e->cfg;
+  const Layout& L = e->lay;
+  const mk::DevModel& m = e->hm;
+  char* ws = e->ws;
+  cudaStream_t st = e->stream;
+  const int H = c.hidden, pw = L.pw, aw = L.aw, pos0 = e->pos;
+  const size_t lo_x = size_t(L.tmax) * H, lo_a = size_t(L.tmax) * aw;  // lo operand offsets
+  const int nh = c.dn_heads, dk = c.dn_dk, dv = c.dn_dv, I = c.mlp;
+  const int nq = c.q_heads, nkv = c.kv_heads, hd = c.head_dim;
+  int32_t* tok = reinterpret_cast<int32_t*>(ws + L.pf_tok);
+  float* X = reinterpret_cast<float*>(ws + L.pf_x);
+  uint16_t* Xn = reinterpret_cast<uint16_t*>(ws + L.pf_xn);
+  float* P = reinterpret_cast<float*>(ws + L.pf_p);
+  float* O = reinterpret_cast<float*>(ws + L.pf_o);
+  uint16_t* A16 = reinterpret_cast<uint16_t*>(ws + L.pf_a16);
+  float* QK = reinterpret_cast<float*>(ws + L.pf_qk);
+  float4* BAK = reinterpret_cast<float4*>(ws + L.pf_bak);
+  cudaError_t r = cudaMemcpyAsync(tok, tokens_host, size_t(T) * 4, cudaMemcpyHostToDevice, st);
+  if (r != cudaSuccess) return cuda_status(r);
+  embed_kernel<<<T, ROW_THREADS, 0, st>>>(tok, m.embed, X, H);
+  e->launches += 1;
+  int rc = MK_OK;
+  for (int l = 0; l < c.n_layers && rc == MK_OK; ++l) {
+    const mk::DevLayer& D = m.layers[l];
+    const mk_engine::LayerMaps& mp = e->maps[l];
+    rmsnorm_bf16_kernel<<<T, ROW_THREADS, 0, st>>>(X, D.attn_norm, Xn, H, c.rms_eps, lo_x);
+    if (!D.is_attn) {
+      rc = launch_gemm(e, mp.in_proj, e->map_xn, P, pw, m.rin, T, H, 0);
+      conv_kernel<<<(m.ch + 255) / 256, 256, 0, st>>>(
+          P, pw, reinterpret_cast<float4*>(m.conv_state[e->cur_buf]) + size_t(D.sub) * m.ch,
+          D.conv_w, m.ch, T);
+      dn_prep_kernel<<<dim3(T, nh), dk, 0, st>>>(P, pw, nh, dk, m.ch, dv, D.A_log, D.dt_bias, QK,
+                                                 BAK, T);
+      float* S = m.dn_state[e->cur_buf] + size_t(D.sub) * nh * dv * dk;
+      const dim3 rgrid(nh, dv / (REC_WARPS * 2));
+      if (dk == 128)
+        recurrence_kernel<128, 2><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, P, pw, 2 * nh * dk,
+                                                                    O, nh * dv, nh, T);
+      else
+        recurrence_kernel<64, 2><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, P, pw, 2 * nh * dk,
+                                                                   O, nh * dv, nh, T);
+      gated_norm_kernel<<<dim3(T, nh), dv, 0, st>>>(O, nh * dv, P, pw, m.ch, D.out_norm, A16, aw,
+                                                    c.rms_eps, lo_a);
+      if (rc == MK_OK) rc = launch_gemm(e, mp.out, e->map_a16_dn, X, H, H, T, nh * dv, 1);
+    } else {
+      rc = launch_gemm(e, mp.q, e->map_xn, P, pw, nq * hd, T, H, 0);
+      if (rc == MK_OK) rc = launch_gemm(e, mp.k, e->map_xn, P + nq * hd, pw, nkv * hd, T, H, 0);
+      if (rc == MK_OK)
+        rc = launch_gemm(e, mp.v, e->map_xn, P + (nq + nkv) * hd, pw, nkv * hd, T, H, 0);
+      const size_t kvo = size_t(D.sub) * nkv * c.max_ctx * hd;
+      rope_kv_kernel<<<dim3(T, nq + nkv), hd / 2, 0, st>>>(P, pw, nq, nkv, hd, m.kc + kvo,
+                                                           m.vc + kvo, c.max_ctx, pos0,
+                                                           c.rope_theta);
+      const dim3 agrid((T + 7) / 8, nq);
+      if (hd == 256)
+        attn_prefill_kernel<256><<<agrid, 256, 0, st>>>(P, pw, m.kc + kvo, m.vc + kvo, c.max_ctx,
+                                                        nq, nkv, pos0, T, A16, aw, lo_a);
+      else if (hd == 128)
+        attn_prefill_kernel<128><<<agrid, 256, 0, st>>>(P, pw, m.kc + kvo, m.vc + kvo, c.max_ctx,
+                                                        nq, nkv, pos0, T, A16, aw, lo_a);
+      else
+        attn_prefill_kernel<64><<<agrid, 256, 0, st>>>(P, pw, m.kc + kvo, m.vc + kvo, c.max_ctx,
+                                                       nq, nkv, pos0, T, A16, aw, lo_a);
+      if (rc == MK_OK) rc = launch_gemm(e, mp.out, e->map_a16_att, X, H, H, T, nq * hd, 1);
+    }
+    rmsnorm_bf16_kernel<<<T, ROW_THREADS, 0, st>>>(X, D.mlp_norm, Xn, H, c.rms_eps, lo_x);
+    if (rc == MK_OK) rc = launch_gemm(e, mp.gate, e->map_xn, P, pw, I, T, H, 0);
+    if (rc == MK_OK) rc = launch_gemm(e, mp.up, e->map_xn, P + I, pw, I, T, H, 0);
+    swiglu_kernel<<<dim3((I + 255) / 256, T), 256, 0, st>>>(P, pw, I, A16, aw, lo_a);
+    if (rc == MK_OK) rc = launch_gemm(e, mp.down, e->map_a16_mlp, X, H, H, T, I, 1);
+    e->launches += D.is_attn ? 5 : 7;  // besides the GEMMs
+  }
+  if (rc != MK_OK) return rc;
+  r = cudaGetLastError();
+  if (r != cudaSuccess) return cuda_status(r);
+  e->pos += T;
   return MK_OK;
 }
 
@@ -344,6 +518,36 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
     delete e;
     return MK_ERR_CUDA;
   }
+  // tensor maps of the prompt path (weights and the chunk's bf16 activations)
+  e->pf_ok = cudaFuncSetAttribute(mk::pf::gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(mk::pf::GEMM_SMEM)) == cudaSuccess;
+  cudaGetLastError();
+  {
+    const int H = c.hidden, T = lay.tmax;
+    const int qd = c.q_heads * c.head_dim, kd = c.kv_heads * c.head_dim;
+    const int vd = c.dn_heads * c.dn_dv;
+    bool ok = e->pf_ok;
+    ok = ok && make_map(&e->map_xn, ws + lay.pf_xn, 2 * T, H, H, mk::pf::BN);
+    ok = ok && make_map(&e->map_a16_dn, ws + lay.pf_a16, 2 * T, vd, lay.aw, mk::pf::BN);
+    ok = ok && make_map(&e->map_a16_mlp, ws + lay.pf_a16, 2 * T, c.mlp, lay.aw, mk::pf::BN);
+    ok = ok && make_map(&e->map_a16_att, ws + lay.pf_a16, 2 * T, qd, lay.aw, mk::pf::BN);
+    for (int l = 0; l < c.n_layers && ok; ++l) {
+      const mk_layer_weights& L = w->layers[l];
+      mk_engine::LayerMaps& mp = e->maps[l];
+      const int BM = mk::pf::BM;
+      ok = make_map(&mp.gate, L.w_gate, c.mlp, H, H, BM) &&
+           make_map(&mp.up, L.w_up, c.mlp, H, H, BM) &&
+           make_map(&mp.down, L.w_down, H, c.mlp, c.mlp, BM);
+      if (ok && c.layer_is_attn[l])
+        ok = make_map(&mp.q, L.w_q, qd, H, H, BM) && make_map(&mp.k, L.w_k, kd, H, H, BM) &&
+             make_map(&mp.v, L.w_v, kd, H, H, BM) && make_map(&mp.out, L.w_o, H, qd, qd, BM);
+      else if (ok)
+        ok = make_map(&mp.in_proj, L.in_proj, m.rin, H, H, BM) &&
+             make_map(&mp.out, L.out_proj, H, vd, vd, BM);
+    }
+    e->pf_ok = ok && (c.dn_dk == 64 || c.dn_dk == 128) && c.dn_dk == c.dn_dv &&
+               (c.head_dim == 64 || c.head_dim == 128 || c.head_dim == 256);
+  }
   int rc = mk_reset(e);
   if (rc != MK_OK) {
     delete e;
@@ -421,7 +625,18 @@ int mk_prefill(mk_engine* e, const int32_t* tokens_host, int n, float* logits_ou
   if (e->pos + n > e->cfg.max_ctx) return MK_ERR_CTX_OVERFLOW;
   for (int i = 0; i < n; ++i)
     if (tokens_host[i] < 0 || tokens_host[i] >= e->cfg.vocab) return MK_ERR_ARG;
-  for (int i = 0; i < n; ++i) {
+  int i = 0;
+  // all but the last position through the tensor-core path, in chunks
+  if (e->pf_ok && n - 1 >= kPrefillMinBatch) {
+    while (i < n - 1) {
+      const int T = (n - 1 - i) < e->lay.tmax ? (n - 1 - i) : e->lay.tmax;
+      const int rc = prefill_chunk(e, tokens_host + i, T);
+      if (rc != MK_OK) return rc;
+      i += T;
+    }
+  }
+  // the rest (at least the last position: its logits and greedy argmax)
+  for (; i < n; ++i) {
     int rc = launch_decode(e, e->pos, e->cur_buf, tokens_host[i], 0,
                            i == n - 1 ? logits_out : nullptr, nullptr);
     if (rc != MK_OK) return rc;
@@ -568,6 +783,33 @@ int mk_delta_step(float* S, const void* q, const void* k, const void* v, const f
     mk::delta_step_kernel<128><<<grid, mk::DS_THREADS, 0, st>>>(S, q16, k16, v16, alpha, beta, o);
   else
     mk::delta_step_kernel<64><<<grid, mk::DS_THREADS, 0, st>>>(S, q16, k16, v16, alpha, beta, o);
+  return cuda_status(cudaGetLastError());
+}
+
+int mk_debug_gemm(const void* W, const void* X, float* C, int n_out, int T, int K,
+                  void* stream) {
+  if (!W || !X || !C || n_out <= 0 || T <= 0 || K <= 0 || K % 64) return MK_ERR_ARG;
+  mk::pf::GemmArgs g;
+  if (!make_map(&g.tw, W, n_out, K, K, mk::pf::BM) ||
+      !make_map(&g.tx, X, 2 * T, K, K, mk::pf::BN))
+    return MK_ERR_UNSUPPORTED;
+  static int* err_word = nullptr;
+  if (!err_word && cudaMalloc(&err_word, 4) != cudaSuccess) return MK_ERR_CUDA;
+  if (cudaFuncSetAttribute(mk::pf::gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(mk::pf::GEMM_SMEM)) != cudaSuccess)
+    return MK_ERR_CUDA;
+  g.c = C;
+  g.ldc = n_out;
+  g.n_out = n_out;
+  g.T = T;
+  g.K = K;
+  g.accumulate = 0;
+  g.x_lo_row = T;
+  g.err = err_word;
+  g.wait_ns = 2000000000LL;
+  const dim3 grid((n_out + mk::pf::BM - 1) / mk::pf::BM, (T + mk::pf::BN - 1) / mk::pf::BN);
+  mk::pf::gemm_tc<<<grid, mk::pf::GEMM_THREADS, mk::pf::GEMM_SMEM,
+                    static_cast<cudaStream_t>(stream)>>>(g);
   return cuda_status(cudaGetLastError());
 }
 

@@ -121,8 +121,17 @@ int mk_reset(mk_engine *e);
 
 /* Run n prompt tokens (host array, values in [0, vocab)) through the stack
  * at positions pos .. pos+n-1 and leave the state and KV cache as n decode
- * steps would.  If logits_out (device, float32 [vocab]) is not NULL it
- * receives the logits of the last prompt position.  n == 0 is a no-op.
+ * steps would, up to rounding (launch post "OS Megakernel that match M5 Max
+ * Tok/w at 2x the Throughput on RTX 3090", results table: prompt processing
+ * "pp520" beside decode).  When n-1 >= 8 the first n-1 positions run as
+ * chunks of up to 1024 positions: every projection one tensor-core GEMM
+ * (bf16 weights; each fp32 activation as a bf16 hi + lo pair; fp32
+ * accumulation), the
+ * causal conv and gated delta rule scanned position by position, causal
+ * attention over cache + chunk.  The last position is always one decode
+ * step, so its logits and greedy argmax come from the decode kernel.
+ * If logits_out (device, float32 [vocab]) is not NULL it receives the
+ * logits of the last prompt position.  n == 0 is a no-op.
  * Errors: MK_ERR_CTX_OVERFLOW when pos+n > max_ctx. */
 int mk_prefill(mk_engine *e, const int32_t *tokens_host, int n,
                float *logits_out);
@@ -207,6 +216,19 @@ int mk_debug_set_wait_limit(mk_engine *e, int64_t limit_ns, int fail_phase);
 int mk_delta_step(float *S, const void *q, const void *k, const void *v,
                   const float *alpha, const float *beta, float *o, int B,
                   int heads, int dk, int dv, void *stream);
+
+/* Debug: the prompt path's tensor-core GEMM on its own, asynchronous on
+ * `stream` (a cudaStream_t, may be NULL):
+ *   C[t][n] = sum_k (X_hi[t][k] + X_lo[t][k]) * W[n][k]
+ *   W device bf16 [n_out][K]; X device bf16 [2][T][K], the hi operands of
+ *   the activations then their lo residuals (an fp32 x is split as
+ *   hi = bf16(x), lo = bf16(x - hi)); C device float32 [T][n_out]; all
+ *   16-byte aligned, K a multiple of 64.
+ * MK_ERR_ARG on bad sizes, MK_ERR_UNSUPPORTED if the TMA descriptors cannot
+ * be encoded.  A device-side wait that runs out is recorded in a word
+ * private to this call (not reported). */
+int mk_debug_gemm(const void *W, const void *X, float *C, int n_out, int T,
+                  int K, void *stream);
 
 /* Human-readable text of a status code. */
 const char *mk_strerror(int status);
