@@ -41,7 +41,7 @@ constexpr int NCT = NCW * 32;           // consumer threads
 constexpr int NTHR = NCT + 32;          // + producer warp
 constexpr int SLOT = 32768;             // ring slot bytes
 constexpr int NSLOT = 6;                // ring slots
-constexpr int ATT_MIN_POS = 64;         // fewest positions per attention split
+constexpr int ATT_MIN_POS = 32;         // fewest positions per attention split
 constexpr int XRAW_MAX = 2048;          // largest hidden size (residual copy in shared memory)
 constexpr int UNION_FLOATS = 4096;      // activation vector | head cache | attention scratch
 constexpr int DN_HEADS_MAX = 4;         // heads one CTA's state rows may touch
@@ -362,90 +362,77 @@ __device__ __forceinline__ bool ll_gather_segs(const LLSeg (&sg)[NSEG], SmemTail
 }
 
 // ----------------------------------------------------------------------------
-// GEMV helpers (warp per row).  Lane l owns 16-byte weight vectors
-// v*32 + l of a row (8 bf16 each) and the matching 8 activation floats.  The
-// vector count per lane NV is a compile-time constant: a runtime bound on the
-// unrolled loop costs more than the arithmetic.
+// GEMV helpers (a warp takes four rows at a time).  Lane l owns 16-byte
+// weight vectors v*32 + l of a row (8 bf16 each) and the matching 8
+// activation floats.
 // ----------------------------------------------------------------------------
-__device__ __forceinline__ void fma8(const uint4 w, const float* x, float& a0, float& a1,
-                                     float& a2, float& a3) {
-  a0 = fmaf(bf_lo(w.x), x[0], a0);
-  a1 = fmaf(bf_hi(w.x), x[1], a1);
-  a2 = fmaf(bf_lo(w.y), x[2], a2);
-  a3 = fmaf(bf_hi(w.y), x[3], a3);
-  a0 = fmaf(bf_lo(w.z), x[4], a0);
-  a1 = fmaf(bf_hi(w.z), x[5], a1);
-  a2 = fmaf(bf_lo(w.w), x[6], a2);
-  a3 = fmaf(bf_hi(w.w), x[7], a3);
+// Two interleaved accumulation chains over one 16-byte weight vector.
+__device__ __forceinline__ void fma8x2(const uint4 w, const float* x, float& a, float& b) {
+  a = fmaf(bf_lo(w.x), x[0], a);
+  b = fmaf(bf_hi(w.x), x[1], b);
+  a = fmaf(bf_lo(w.y), x[2], a);
+  b = fmaf(bf_hi(w.y), x[3], b);
+  a = fmaf(bf_lo(w.z), x[4], a);
+  b = fmaf(bf_hi(w.z), x[5], b);
+  a = fmaf(bf_lo(w.w), x[6], a);
+  b = fmaf(bf_hi(w.w), x[7], b);
 }
 
-// PRED: the row has fewer than 32 vectors (small models), lanes past nvec idle.
-template <int NV, bool PRED>
-__device__ __forceinline__ void load_x(float (&xr)[NV][8], const float* xs, int nvec, int lane) {
-#pragma unroll
-  for (int v = 0; v < NV; ++v) {
-    const int idx = v * 32 + lane;
-    if (!PRED || idx < nvec) {
-      const float4 p = reinterpret_cast<const float4*>(xs)[idx * 2];
-      const float4 q = reinterpret_cast<const float4*>(xs)[idx * 2 + 1];
-      xr[v][0] = p.x; xr[v][1] = p.y; xr[v][2] = p.z; xr[v][3] = p.w;
-      xr[v][4] = q.x; xr[v][5] = q.y; xr[v][6] = q.z; xr[v][7] = q.w;
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) xr[v][e] = 0.f;
-    }
+// This lane's partial dot products of four rows (in shared memory) with the
+// activation (shared memory): lane l takes 16-byte vectors l, l+32, ... of
+// each row and the matching 8 activation floats, read once for the four
+// rows.  One runtime loop serves every row length: the kernel runs each
+// phase's code once per token, so a compact instruction footprint beats
+// per-length unrolled copies.
+__device__ __forceinline__ void dot4(const unsigned char* r0, const unsigned char* r1,
+                                     const unsigned char* r2, const unsigned char* r3,
+                                     const float* xs, int nvec, int lane, float (&acc)[4]) {
+  const uint4* w0 = reinterpret_cast<const uint4*>(r0);
+  const uint4* w1 = reinterpret_cast<const uint4*>(r1);
+  const uint4* w2 = reinterpret_cast<const uint4*>(r2);
+  const uint4* w3 = reinterpret_cast<const uint4*>(r3);
+  float s[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+  for (int idx = lane; idx < nvec; idx += 32) {
+    const float4 p = reinterpret_cast<const float4*>(xs)[idx * 2];
+    const float4 q = reinterpret_cast<const float4*>(xs)[idx * 2 + 1];
+    const float x[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
+    const uint4 u0 = w0[idx], u1 = w1[idx], u2 = w2[idx], u3 = w3[idx];
+    fma8x2(u0, x, s[0][0], s[0][1]);
+    fma8x2(u1, x, s[1][0], s[1][1]);
+    fma8x2(u2, x, s[2][0], s[2][1]);
+    fma8x2(u3, x, s[3][0], s[3][1]);
   }
-}
-
-template <int NV, bool PRED>
-__device__ __forceinline__ float dot_x(const unsigned char* row, const float (&xr)[NV][8],
-                                       int nvec, int lane) {
-  const uint4* w = reinterpret_cast<const uint4*>(row);
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-  for (int v = 0; v < NV; ++v) {
-    const int idx = v * 32 + lane;
-    if (!PRED || idx < nvec) fma8(w[idx], xr[v], a0, a1, a2, a3);
-  }
-  return (a0 + a1) + (a2 + a3);
+  for (int q = 0; q < 4; ++q) acc[q] = s[q][0] + s[q][1];
 }
 
-__device__ __forceinline__ void fma8_xs(const uint4 w, const float* xs, int idx, float& a0,
-                                        float& a1, float& a2, float& a3) {
-  float x[8];
-  const float4 p = reinterpret_cast<const float4*>(xs)[idx * 2];
-  const float4 q = reinterpret_cast<const float4*>(xs)[idx * 2 + 1];
-  x[0] = p.x; x[1] = p.y; x[2] = p.z; x[3] = p.w;
-  x[4] = q.x; x[5] = q.y; x[6] = q.z; x[7] = q.w;
-  fma8(w, x, a0, a1, a2, a3);
-}
-
-// Activation read from shared memory (rows too long for registers).  NV > 0:
-// exactly NV vectors per lane; NV == 0: any length (runtime loop).
-template <int NV>
-__device__ __forceinline__ float dot_xs(const unsigned char* row, const float* xs, int nvec,
-                                        int lane) {
-  const uint4* w = reinterpret_cast<const uint4*>(row);
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-  if constexpr (NV > 0) {
-#pragma unroll
-    for (int v = 0; v < NV; ++v) fma8_xs(w[v * 32 + lane], xs, v * 32 + lane, a0, a1, a2, a3);
-  } else {
-    for (int idx = lane; idx < nvec; idx += 32) fma8_xs(w[idx], xs, idx, a0, a1, a2, a3);
-  }
-  return (a0 + a1) + (a2 + a3);
+// Warp reduction of four values at once (6 shuffles instead of 20): on
+// return lanes 8q .. 8q+7 hold the warp-wide sum of input q.
+__device__ __forceinline__ float reduce4(float a, float b, float c, float d, int lane) {
+  const bool h16 = (lane & 16) != 0;
+  float x0 = h16 ? c : a, x1 = h16 ? d : b;
+  const float y0 = h16 ? a : c, y1 = h16 ? b : d;
+  x0 += __shfl_xor_sync(0xffffffffu, y0, 16);
+  x1 += __shfl_xor_sync(0xffffffffu, y1, 16);
+  const bool h8 = (lane & 8) != 0;
+  float z = h8 ? x1 : x0;
+  const float w = h8 ? x0 : x1;
+  z += __shfl_xor_sync(0xffffffffu, w, 8);
+  z += __shfl_xor_sync(0xffffffffu, z, 4);
+  z += __shfl_xor_sync(0xffffffffu, z, 2);
+  z += __shfl_xor_sync(0xffffffffu, z, 1);
+  return z;
 }
 
 // ---- matrix phases ------------------------------------------------------------
-// One out-of-line routine serves every matrix phase, so the hot loop exists
-// once in the instruction stream (a phase switch then finds it cached); the
-// epilogue is a small runtime switch.
+// One routine serves every matrix phase, so the hot loop exists once in the
+// instruction stream (a phase switch then finds it cached); the epilogue is a
+// small runtime switch.
 enum EpiKind { EPI_STORE, EPI_RESID, EPI_INPROJ, EPI_SWIGLU, EPI_LOGITS };
 
 struct GemvJob {
   PD d;
   int epi;                   // EpiKind
-  int shape;                 // GemvShape of the row length
   unsigned long long* dst;   // tagged destination, indexed by row
   const float* xraw;         // EPI_RESID: residual before the update (shared memory)
   float* hidden;             // EPI_RESID: optional per-layer dump
@@ -496,11 +483,13 @@ __device__ __forceinline__ void gemv_epilogue(const GemvJob& j, int row, float y
 }
 
 // Walk the CTA's chunks of one matrix phase.  Each warp takes its rows of a
-// chunk two at a time (independent reductions overlap); for EPI_SWIGLU the
-// pair is a gate row (plane 0) and the matching up row (plane 1).  NV/PRED/XS
-// select the activation layout (see dot_x / dot_xs).  Returns the chunk
-// counter after the phase.
-template <int NV, bool PRED, bool XS>
+// chunk four at a time (rows i, i+NCW, i+2NCW, i+3NCW; for EPI_SWIGLU the
+// gate and up rows of i and i+NCW), reduces the four dot products in one
+// transposed shuffle tree and parks each result in lane (count of results
+// so far); the epilogue then runs once per 32 results with every lane
+// finishing its own row, instead of one lane finishing rows one by one.
+// The activation vector is in shared memory (xs).  Returns the chunk counter
+// after the phase.
 __device__ __forceinline__ uint32_t gemv_core(const GemvJob& j, uint32_t g, unsigned char* ring,
                                               SmemTail* t, int* err, long long wait_ns,
                                               const float* xs) {
@@ -508,11 +497,10 @@ __device__ __forceinline__ uint32_t gemv_core(const GemvJob& j, uint32_t g, unsi
   const PD& d = j.d;
   const int nvec = int(d.row_bytes / 16);
   const bool swiglu = j.epi == EPI_SWIGLU;
-  constexpr int NR = XS ? 1 : NV;
-  float xr[NR][8];
-  if constexpr (!XS) load_x<NV, PRED>(xr, xs, nvec, lane);
   float best_v = -INFINITY;
   int best_i = 0x7FFFFFFF;
+  float kv = 0.f, kv2 = 0.f;  // parked result (and up value for EPI_SWIGLU) of this lane
+  int krow = 0, nb = 0;       // its row; number of parked results in the warp
   int local = 0;
 #pragma unroll 1
   for (int r = d.r0; r < d.r0 + d.n; r += d.rpc, ++g, local += d.rpc) {
@@ -520,86 +508,87 @@ __device__ __forceinline__ uint32_t gemv_core(const GemvJob& j, uint32_t g, unsi
     if (bounded_wait(&t->full[slot], (g / NSLOT) & 1, t, err, wait_ns)) {
       const int nr = min(d.rpc, d.r0 + d.n - r);
       const unsigned char* base = ring + size_t(slot) * SLOT;
-      const int step = swiglu ? NCW : 2 * NCW;
+      const size_t rb = d.row_bytes;
+      const int step = swiglu ? 2 * NCW : 4 * NCW;
 #pragma unroll 1
       for (int i = (warp - (local % NCW) + NCW) % NCW; i < nr; i += step) {
-        // rows a and b: (i, i + NCW) of plane 0, or (i of plane 0, i of plane 1)
-        const int ib = swiglu ? i : i + NCW;
-        const bool hb = swiglu || ib < nr;
-        const unsigned char* ra = base + size_t(i) * d.row_bytes;
-        const unsigned char* rb = base + size_t(swiglu ? d.rpc + i : ib) * d.row_bytes;
-        float pa, pb = 0.f;
-        if constexpr (XS) {
-          pa = dot_xs<NV>(ra, xs, nvec, lane);
-          if (hb) pb = dot_xs<NV>(rb, xs, nvec, lane);
+        int nout;
+        const unsigned char *p0, *p1, *p2, *p3;
+        if (swiglu) {
+          nout = i + NCW < nr ? 2 : 1;
+          const int i1 = nout > 1 ? i + NCW : i;
+          p0 = base + size_t(i) * rb;
+          p1 = base + size_t(d.rpc + i) * rb;
+          p2 = base + size_t(i1) * rb;
+          p3 = base + size_t(d.rpc + i1) * rb;
         } else {
-          pa = dot_x<NV, PRED>(ra, xr, nvec, lane);
-          if (hb) pb = dot_x<NV, PRED>(rb, xr, nvec, lane);
+          nout = min(4, (nr - i + NCW - 1) / NCW);
+          p0 = base + size_t(i) * rb;
+          p1 = base + size_t(nout > 1 ? i + NCW : i) * rb;
+          p2 = base + size_t(nout > 2 ? i + 2 * NCW : i) * rb;
+          p3 = base + size_t(nout > 3 ? i + 3 * NCW : i) * rb;
         }
-        pa = warp_sum(pa);
-        pb = warp_sum(pb);
-        if (lane == 0) {
-          if (swiglu) {
-            gemv_epilogue(j, r + i, pa, pb, best_v, best_i);
-          } else {
-            gemv_epilogue(j, r + i, pa, 0.f, best_v, best_i);
-            if (hb) gemv_epilogue(j, r + ib, pb, 0.f, best_v, best_i);
+        float acc[4];
+        dot4(p0, p1, p2, p3, xs, nvec, lane, acc);
+        const float z = reduce4(acc[0], acc[1], acc[2], acc[3], lane);
+        if (nb + nout > 32) {
+          if (lane < nb) gemv_epilogue(j, krow, kv, kv2, best_v, best_i);
+          nb = 0;
+        }
+        const int q = lane - nb;
+        if (swiglu) {
+          const float gv = __shfl_sync(0xffffffffu, z, (q & 1) << 4);
+          const float uv = __shfl_sync(0xffffffffu, z, ((q & 1) << 4) + 8);
+          if (q >= 0 && q < nout) {
+            kv = gv;
+            kv2 = uv;
+            krow = r + i + q * NCW;
+          }
+        } else {
+          const float v = __shfl_sync(0xffffffffu, z, (q & 3) << 3);
+          if (q >= 0 && q < nout) {
+            kv = v;
+            krow = r + i + q * NCW;
           }
         }
+        nb += nout;
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&t->empty[slot]);
   }
-  if (j.epi == EPI_LOGITS && lane == 0 && best_i != 0x7FFFFFFF)
+  if (lane < nb) gemv_epilogue(j, krow, kv, kv2, best_v, best_i);
+  if (j.epi == EPI_LOGITS && best_i != 0x7FFFFFFF)
     atomicMax(&t->best, pack_argmax(best_v, best_i));
   return g;
-}
-
-// Activation layouts the kernel instantiates (chosen from the row length K,
-// a multiple of 8): fewer than 32 vectors (predicated), 1/2/3/4/8 vectors per
-// lane in registers, 14 per lane from shared memory, anything else from
-// shared memory with a runtime loop.
-enum GemvShape { GS_PRED1 = 0, GS_R1, GS_R2, GS_R3, GS_R4, GS_R8, GS_S14, GS_SANY };
-
-__host__ __device__ constexpr int gemv_shape(int K) {
-  return (K / 8) < 32        ? GS_PRED1
-         : (K / 8) % 32 != 0 ? GS_SANY
-         : (K / 256) == 1    ? GS_R1
-         : (K / 256) == 2    ? GS_R2
-         : (K / 256) == 3    ? GS_R3
-         : (K / 256) == 4    ? GS_R4
-         : (K / 256) == 8    ? GS_R8
-         : (K / 256) == 14   ? GS_S14
-                             : GS_SANY;
-}
-
-__device__ __forceinline__ uint32_t gemv_dispatch(const GemvJob& j, uint32_t g,
-                                                  unsigned char* ring, SmemTail* t, int* err,
-                                                  long long wait_ns, const float* xs) {
-  switch (j.shape) {
-    case GS_PRED1: return gemv_core<1, true, false>(j, g, ring, t, err, wait_ns, xs);
-    case GS_R1: return gemv_core<1, false, false>(j, g, ring, t, err, wait_ns, xs);
-    case GS_R2: return gemv_core<2, false, false>(j, g, ring, t, err, wait_ns, xs);
-    case GS_R3: return gemv_core<3, false, false>(j, g, ring, t, err, wait_ns, xs);
-    case GS_R4: return gemv_core<4, false, false>(j, g, ring, t, err, wait_ns, xs);
-    case GS_R8: return gemv_core<8, false, false>(j, g, ring, t, err, wait_ns, xs);
-    case GS_S14: return gemv_core<14, false, true>(j, g, ring, t, err, wait_ns, xs);
-    default: return gemv_core<0, false, true>(j, g, ring, t, err, wait_ns, xs);
-  }
 }
 
 // ----------------------------------------------------------------------------
 // RMSNorm of the vector already in `xin` (all NCT consumer threads):
 // xin = xin * rsqrt(mean(xin^2) + eps) * gain, keeping the raw copy in xraw.
 // ----------------------------------------------------------------------------
-__device__ __forceinline__ void rmsnorm_inplace(float* xin, float* xraw, const uint16_t* gain,
+// Gains of RMSNorm as this thread uses them (element tid + k*NCT), loaded
+// before the input is awaited so their latency overlaps the wait.
+constexpr int GK = per_thread(XRAW_MAX);
+__device__ __forceinline__ void load_gains(float (&gv)[GK], const uint16_t* gain, int H, int tid) {
+#pragma unroll
+  for (int k = 0; k < GK; ++k) {
+    const int i = tid + k * NCT;
+    gv[k] = (gain && i < H) ? bf2f(gain[i]) : 1.f;
+  }
+}
+
+__device__ __forceinline__ void rmsnorm_inplace(float* xin, float* xraw, const float (&gv)[GK],
                                                 int H, float eps, SmemTail* t, int tid) {
   float ss = 0.f;
-  for (int i = tid; i < H; i += NCT) {
-    const float v = xin[i];
-    if (xraw) xraw[i] = v;
-    ss = fmaf(v, v, ss);
+#pragma unroll
+  for (int k = 0; k < GK; ++k) {
+    const int i = tid + k * NCT;
+    if (i < H) {
+      const float v = xin[i];
+      if (xraw) xraw[i] = v;
+      ss = fmaf(v, v, ss);
+    }
   }
   ss = warp_sum(ss);
   if ((tid & 31) == 0) t->red[tid >> 5] = ss;
@@ -608,7 +597,11 @@ __device__ __forceinline__ void rmsnorm_inplace(float* xin, float* xraw, const u
 #pragma unroll
   for (int w = 0; w < NCW; ++w) tot += t->red[w];
   const float inv = 1.0f / sqrtf(tot / float(H) + eps);
-  for (int i = tid; i < H; i += NCT) xin[i] = xin[i] * inv * bf2f(gain[i]);
+#pragma unroll
+  for (int k = 0; k < GK; ++k) {
+    const int i = tid + k * NCT;
+    if (i < H) xin[i] = xin[i] * inv * gv[k];
+  }
   named_sync(1, NCT);
 }
 
@@ -741,15 +734,33 @@ template <int G, int EPL>
 __device__ __forceinline__ void att_consume(float (&am)[G], float (&al)[G], float (&acc)[G][EPL],
                                             const float (&qr)[G][EPL], const float* kf,
                                             const float* vf, float scale) {
+  float sc[G];
+  if constexpr (G == 4) {
+    // the four heads' scores reduced together, then broadcast from lane 8j
+    float pz[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      pz[j] = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) pz[j] = fmaf(qr[j][e], kf[e], pz[j]);
+    }
+    const float z = reduce4(pz[0], pz[1], pz[2], pz[3], threadIdx.x & 31);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sc[j] = __shfl_sync(0xffffffffu, z, 8 * j) * scale;
+  } else {
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) s = fmaf(qr[j][e], kf[e], s);
+      sc[j] = warp_sum(s) * scale;
+    }
+  }
 #pragma unroll
   for (int j = 0; j < G; ++j) {
-    float s = 0.f;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) s = fmaf(qr[j][e], kf[e], s);
-    s = warp_sum(s) * scale;
-    const float mn = fmaxf(am[j], s);
+    const float mn = fmaxf(am[j], sc[j]);
     const float corr = expf(am[j] - mn);
-    const float pr = expf(s - mn);
+    const float pr = expf(sc[j] - mn);
     al[j] = al[j] * corr + pr;
 #pragma unroll
     for (int e = 0; e < EPL; ++e) acc[j][e] = fmaf(pr, vf[e], acc[j][e] * corr);
@@ -967,7 +978,7 @@ __device__ __forceinline__ void attention_phase(const DevModel& M, const StepArg
 // Cursor over one CTA's chunk schedule for one launch: every phase of every
 // layer, then the LM head, each split into chunks of at most `rpc` rows.
 // ----------------------------------------------------------------------------
-constexpr size_t PF_AHEAD = size_t(256) << 10;  // L2 prefetch distance per CTA (bytes)
+constexpr size_t PF_AHEAD = size_t(128) << 10;  // L2 prefetch distance per CTA (bytes)
 
 struct ChunkCursor {
   int l, p, np, gp;
@@ -1153,6 +1164,10 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
           float4* conv_s = reinterpret_cast<float4*>(uni + 2048);
           uint2* conv_taps = reinterpret_cast<uint2*>(uni + 2048 + 4 * CONV_ROWS_MAX);
           float4* conv_g = reinterpret_cast<float4*>(M.conv_state[a.st_buf]) + size_t(L.sub) * M.ch;
+          const uint16_t* gain = kind == PH_GU ? L.mlp_norm
+                                 : kind == PH_LM ? M.final_norm : L.attn_norm;
+          float gv[GK];
+          load_gains(gv, gain, M.H, tid);
           if (!dry) {
             if (kind == PH_DN_IN) {
               // stage the conv history and taps of this CTA's q|k|v rows first
@@ -1171,13 +1186,9 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
             }
           }
           const bool bad = named_sync_or(1, NCT, !ok);
-          if (!dry && !bad) {
-            const uint16_t* gain = kind == PH_GU ? L.mlp_norm
-                                   : kind == PH_LM ? M.final_norm : L.attn_norm;
-            rmsnorm_inplace(uni, kind == PH_LM ? nullptr : xraw, gain, M.H, M.eps, t, tid);
-          }
+          if (!dry && !bad)
+            rmsnorm_inplace(uni, kind == PH_LM ? nullptr : xraw, gv, M.H, M.eps, t, tid);
           gemv = true;
-          j.shape = gemv_shape(M.H);
           if (kind == PH_DN_IN) {
             j.epi = EPI_INPROJ;
             j.dst = M.inp_ll;
@@ -1203,7 +1214,6 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
         case PH_K:
         case PH_V: {
           gemv = true;
-          j.shape = gemv_shape(M.H);
           j.epi = EPI_STORE;
           j.dst = M.qkv_ll + (kind == PH_K ? M.nq * HD : (M.nq + M.nkv) * HD);
           if (kind == PH_K) tag_k = tag_me;
@@ -1213,6 +1223,10 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
         case PH_OUT: {
           bool ok = true;
           const int K = L.is_attn ? M.nq * M.hd : M.nh * M.dv;
+          constexpr int EPL_G = DK / 32;  // gated-norm elements per lane (dv == dk)
+          float gw[EPL_G];
+#pragma unroll
+          for (int e = 0; e < EPL_G; ++e) gw[e] = L.is_attn ? 0.f : bf2f(L.out_norm[lane * EPL_G + e]);
           if (!dry) {
             if (L.is_attn) {
               ok = ll_gather<per_thread(UNION_FLOATS)>(uni, M.atto_ll, K, tag_att | dbg, t, M.err,
@@ -1243,14 +1257,12 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
 #pragma unroll
               for (int e = 0; e < EPL; ++e) {
                 const int i = lane * EPL + e;
-                uni[h * DK + i] =
-                    o[e] * inv * bf2f(L.out_norm[i]) * siluf_(uni[2048 + h * DK + i]);
+                uni[h * DK + i] = o[e] * inv * gw[e] * siluf_(uni[2048 + h * DK + i]);
               }
             }
             named_sync(1, NCT);
           }
           gemv = true;
-          j.shape = gemv_shape(K);
           j.epi = EPI_RESID;
           j.dst = M.x_ll + size_t(xb ^ 1) * M.H;
           j.xraw = xraw;
@@ -1265,7 +1277,6 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
                                                      a.wait_ns, tid);
           named_sync_or(1, NCT, !ok);
           gemv = true;
-          j.shape = gemv_shape(M.I);
           j.epi = EPI_RESID;
           j.dst = M.x_ll + size_t(xb ^ 1) * M.H;
           j.xraw = xraw;
@@ -1287,7 +1298,7 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
         default:
           break;
       }
-      if (gemv) g = gemv_dispatch(j, g, ring, t, M.err, a.wait_ns, uni);
+      if (gemv) g = gemv_core(j, g, ring, t, M.err, a.wait_ns, uni);
     }
   }
 

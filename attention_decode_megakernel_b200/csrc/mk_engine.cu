@@ -26,7 +26,7 @@ struct Layout {
   size_t x, inp, dno, qkv, atto, mlph, part, hidden, logits, tickets, err, amax;
   // multi-token prompt path: T_MAX positions per chunk
   int tmax, pw, aw;
-  size_t pf_tok, pf_x, pf_xn, pf_p, pf_o, pf_a16, pf_qk, pf_bak;
+  size_t pf_tok, pf_x, pf_xn, pf_p, pf_o, pf_a16, pf_qk, pf_bak, pf_att;
   size_t total;
 };
 
@@ -103,6 +103,9 @@ Layout make_layout(const mk_config& c) {
     L.pf_a16 = take(size_t(2) * T * aw * 2);  // [hi|lo][T][aw] bf16
     L.pf_qk = take(size_t(c.dn_heads) * T * 2 * c.dn_dk * 4);
     L.pf_bak = take(size_t(c.dn_heads) * T * 16);
+    // key-split attention partials of a short chunk: [t][q head][range][hd + 2]
+    const size_t nsplit = (size_t(c.max_ctx) + mk::pf::ATT_SPLIT_LEN - 1) / mk::pf::ATT_SPLIT_LEN;
+    L.pf_att = take(size_t(mk::kMaxVerify) * c.q_heads * nsplit * (c.head_dim + 2) * 4);
   }
   L.total = off;
   return L;
@@ -195,7 +198,7 @@ struct mk_engine {
   struct LayerMaps {
     CUtensorMap in_proj, out, q, k, v, gate, up, down;
   } maps[MK_MAX_LAYERS];
-  CUtensorMap map_xn, map_a16_dn, map_a16_mlp, map_a16_att;
+  CUtensorMap map_xn, map_a16_dn, map_a16_mlp, map_a16_att, map_embed;
 };
 
 namespace {
@@ -247,8 +250,21 @@ int launch_decode(mk_engine* e, int pos, int st_buf, int token, int tok_src, flo
   return MK_OK;
 }
 
+// One tensor-core GEMM launch.  For a chunk of at most one token tile with
+// few output tiles (verify), K is split over gridDim.z so every SM streams
+// weights; the partial sums are added atomically, so a non-accumulating
+// output is zeroed first.
 int launch_gemm(mk_engine* e, const CUtensorMap& tw, const CUtensorMap& tx, float* c, int ldc,
                 int n_out, int T, int K, int accumulate) {
+  const int tiles = ((n_out + mk::pf::BM - 1) / mk::pf::BM) * ((T + mk::pf::BN - 1) / mk::pf::BN);
+  int ks = T <= mk::pf::BN ? (e->ncta + tiles - 1) / tiles : 1;  // short chunks only
+  if (ks > K / mk::pf::BK) ks = K / mk::pf::BK;
+  if (ks < 1) ks = 1;
+  if (ks > 1 && !accumulate) {
+    const cudaError_t r =
+        cudaMemset2DAsync(c, size_t(ldc) * 4, 0, size_t(n_out) * 4, T, e->stream);
+    if (r != cudaSuccess) return cuda_status(r);
+  }
   mk::pf::GemmArgs g;
   g.tw = tw;
   g.tx = tx;
@@ -259,16 +275,22 @@ int launch_gemm(mk_engine* e, const CUtensorMap& tw, const CUtensorMap& tx, floa
   g.K = K;
   g.accumulate = accumulate;
   g.x_lo_row = e->lay.tmax;
+  g.k_split = ks;
   g.err = e->hm.err;
   g.wait_ns = e->wait_ns;
-  const dim3 grid((n_out + mk::pf::BM - 1) / mk::pf::BM, (T + mk::pf::BN - 1) / mk::pf::BN);
+  const dim3 grid((n_out + mk::pf::BM - 1) / mk::pf::BM, (T + mk::pf::BN - 1) / mk::pf::BN, ks);
   mk::pf::gemm_tc<<<grid, mk::pf::GEMM_THREADS, mk::pf::GEMM_SMEM, e->stream>>>(g);
   e->launches += 1;
   return cuda_status(cudaGetLastError());
 }
 
-// The stack over T prompt positions starting at e->pos (no logits).
-int prefill_chunk(mk_engine* e, const int32_t* tokens_host, int T) {
+// The stack over T positions starting at e->pos through the chunk kernels.
+// Prompt chunk (ck_bufs == nullptr): the state is updated in place and the
+// position advances.  Verify chunk: the state after position t goes to state
+// buffer ck_bufs[t], the current state is left as it was, the position does
+// not move, and logits_out [T][vocab] receives every position's logits.
+int run_chunk(mk_engine* e, const int32_t* tokens_host, int T, const int* ck_bufs,
+              float* logits_out) {
   using namespace mk::pf;
   const mk_config& c = e->cfg;
   const Layout& L = e->lay;
@@ -298,19 +320,25 @@ int prefill_chunk(mk_engine* e, const int32_t* tokens_host, int T) {
     rmsnorm_bf16_kernel<<<T, ROW_THREADS, 0, st>>>(X, D.attn_norm, Xn, H, c.rms_eps, lo_x);
     if (!D.is_attn) {
       rc = launch_gemm(e, mp.in_proj, e->map_xn, P, pw, m.rin, T, H, 0);
+      mk::pf::Ckpt ckc{}, cks{};
+      if (ck_bufs)
+        for (int t = 0; t < T; ++t) {
+          ckc.p[t] = m.conv_state[ck_bufs[t]] + size_t(D.sub) * m.ch * 4;
+          cks.p[t] = m.dn_state[ck_bufs[t]] + size_t(D.sub) * nh * dv * dk;
+        }
       conv_kernel<<<(m.ch + 255) / 256, 256, 0, st>>>(
           P, pw, reinterpret_cast<float4*>(m.conv_state[e->cur_buf]) + size_t(D.sub) * m.ch,
-          D.conv_w, m.ch, T);
+          D.conv_w, m.ch, T, ckc);
       dn_prep_kernel<<<dim3(T, nh), dk, 0, st>>>(P, pw, nh, dk, m.ch, dv, D.A_log, D.dt_bias, QK,
                                                  BAK, T);
       float* S = m.dn_state[e->cur_buf] + size_t(D.sub) * nh * dv * dk;
       const dim3 rgrid(nh, dv / (REC_WARPS * 2));
       if (dk == 128)
         recurrence_kernel<128, 2><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, P, pw, 2 * nh * dk,
-                                                                    O, nh * dv, nh, T);
+                                                                    O, nh * dv, nh, T, cks);
       else
         recurrence_kernel<64, 2><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, P, pw, 2 * nh * dk,
-                                                                   O, nh * dv, nh, T);
+                                                                   O, nh * dv, nh, T, cks);
       gated_norm_kernel<<<dim3(T, nh), dv, 0, st>>>(O, nh * dv, P, pw, m.ch, D.out_norm, A16, aw,
                                                     c.rms_eps, lo_a);
       if (rc == MK_OK) rc = launch_gemm(e, mp.out, e->map_a16_dn, X, H, H, T, nh * dv, 1);
@@ -323,16 +351,41 @@ int prefill_chunk(mk_engine* e, const int32_t* tokens_host, int T) {
       rope_kv_kernel<<<dim3(T, nq + nkv), hd / 2, 0, st>>>(P, pw, nq, nkv, hd, m.kc + kvo,
                                                            m.vc + kvo, c.max_ctx, pos0,
                                                            c.rope_theta);
-      const dim3 agrid((T + 7) / 8, nq);
-      if (hd == 256)
-        attn_prefill_kernel<256><<<agrid, 256, 0, st>>>(P, pw, m.kc + kvo, m.vc + kvo, c.max_ctx,
-                                                        nq, nkv, pos0, T, A16, aw, lo_a);
-      else if (hd == 128)
-        attn_prefill_kernel<128><<<agrid, 256, 0, st>>>(P, pw, m.kc + kvo, m.vc + kvo, c.max_ctx,
-                                                        nq, nkv, pos0, T, A16, aw, lo_a);
-      else
-        attn_prefill_kernel<64><<<agrid, 256, 0, st>>>(P, pw, m.kc + kvo, m.vc + kvo, c.max_ctx,
-                                                       nq, nkv, pos0, T, A16, aw, lo_a);
+      if (T <= mk::kMaxVerify) {
+        // few queries: split the keys too, then merge the ranges
+        float* part = reinterpret_cast<float*>(ws + L.pf_att);
+        const int nsplit = (pos0 + T + ATT_SPLIT_LEN - 1) / ATT_SPLIT_LEN;
+        const dim3 sg((nsplit + ATT_SPLIT_WARPS - 1) / ATT_SPLIT_WARPS, nq, T);
+        const dim3 mg(nq, T);
+        if (hd == 256) {
+          attn_split_kernel<256><<<sg, ATT_SPLIT_WARPS * 32, 0, st>>>(
+              P, pw, m.kc + kvo, m.vc + kvo, c.max_ctx, nq, nkv, pos0, nsplit, part);
+          attn_merge_kernel<256><<<mg, 256, 0, st>>>(part, nq, nsplit, A16, aw, lo_a);
+        } else if (hd == 128) {
+          attn_split_kernel<128><<<sg, ATT_SPLIT_WARPS * 32, 0, st>>>(
+              P, pw, m.kc + kvo, m.vc + kvo, c.max_ctx, nq, nkv, pos0, nsplit, part);
+          attn_merge_kernel<128><<<mg, 128, 0, st>>>(part, nq, nsplit, A16, aw, lo_a);
+        } else {
+          attn_split_kernel<64><<<sg, ATT_SPLIT_WARPS * 32, 0, st>>>(
+              P, pw, m.kc + kvo, m.vc + kvo, c.max_ctx, nq, nkv, pos0, nsplit, part);
+          attn_merge_kernel<64><<<mg, 64, 0, st>>>(part, nq, nsplit, A16, aw, lo_a);
+        }
+        e->launches += 1;  // the merge
+      } else {
+        const dim3 agrid((T + 7) / 8, nq);
+        if (hd == 256)
+          attn_prefill_kernel<256><<<agrid, 256, 0, st>>>(P, pw, m.kc + kvo, m.vc + kvo,
+                                                          c.max_ctx, nq, nkv, pos0, T, A16, aw,
+                                                          lo_a);
+        else if (hd == 128)
+          attn_prefill_kernel<128><<<agrid, 256, 0, st>>>(P, pw, m.kc + kvo, m.vc + kvo,
+                                                          c.max_ctx, nq, nkv, pos0, T, A16, aw,
+                                                          lo_a);
+        else
+          attn_prefill_kernel<64><<<agrid, 256, 0, st>>>(P, pw, m.kc + kvo, m.vc + kvo,
+                                                         c.max_ctx, nq, nkv, pos0, T, A16, aw,
+                                                         lo_a);
+      }
       if (rc == MK_OK) rc = launch_gemm(e, mp.out, e->map_a16_att, X, H, H, T, nq * hd, 1);
     }
     rmsnorm_bf16_kernel<<<T, ROW_THREADS, 0, st>>>(X, D.mlp_norm, Xn, H, c.rms_eps, lo_x);
@@ -343,9 +396,16 @@ int prefill_chunk(mk_engine* e, const int32_t* tokens_host, int T) {
     e->launches += D.is_attn ? 5 : 7;  // besides the GEMMs
   }
   if (rc != MK_OK) return rc;
+  if (logits_out) {
+    // final norm and the tied LM head for every position of the chunk
+    rmsnorm_bf16_kernel<<<T, ROW_THREADS, 0, st>>>(X, m.final_norm, Xn, H, c.rms_eps, lo_x);
+    e->launches += 1;
+    rc = launch_gemm(e, e->map_embed, e->map_xn, logits_out, c.vocab, c.vocab, T, H, 0);
+    if (rc != MK_OK) return rc;
+  }
   r = cudaGetLastError();
   if (r != cudaSuccess) return cuda_status(r);
-  e->pos += T;
+  if (!ck_bufs) e->pos += T;
   return MK_OK;
 }
 
@@ -528,6 +588,7 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
     const int vd = c.dn_heads * c.dn_dv;
     bool ok = e->pf_ok;
     ok = ok && make_map(&e->map_xn, ws + lay.pf_xn, 2 * T, H, H, mk::pf::BN);
+    ok = ok && make_map(&e->map_embed, w->embed, c.vocab, H, H, mk::pf::BM);
     ok = ok && make_map(&e->map_a16_dn, ws + lay.pf_a16, 2 * T, vd, lay.aw, mk::pf::BN);
     ok = ok && make_map(&e->map_a16_mlp, ws + lay.pf_a16, 2 * T, c.mlp, lay.aw, mk::pf::BN);
     ok = ok && make_map(&e->map_a16_att, ws + lay.pf_a16, 2 * T, qd, lay.aw, mk::pf::BN);
@@ -630,7 +691,7 @@ int mk_prefill(mk_engine* e, const int32_t* tokens_host, int n, float* logits_ou
   if (e->pf_ok && n - 1 >= kPrefillMinBatch) {
     while (i < n - 1) {
       const int T = (n - 1 - i) < e->lay.tmax ? (n - 1 - i) : e->lay.tmax;
-      const int rc = prefill_chunk(e, tokens_host + i, T);
+      const int rc = run_chunk(e, tokens_host + i, T, nullptr, nullptr);
       if (rc != MK_OK) return rc;
       i += T;
     }
@@ -651,6 +712,15 @@ int mk_verify(mk_engine* e, const int32_t* tokens_host, int n, float* logits_out
   if (e->pos + n > e->cfg.max_ctx) return MK_ERR_CTX_OVERFLOW;
   for (int i = 0; i < n; ++i)
     if (tokens_host[i] < 0 || tokens_host[i] >= e->cfg.vocab) return MK_ERR_ARG;
+  if (e->pf_ok) {
+    // one chunk: every projection a tensor-core GEMM over the n positions,
+    // the scans writing the state after each position to its own buffer
+    for (int j = 0; j < n; ++j) e->verify_bufs[j] = (e->cur_buf + 1 + j) % mk::kStateBufs;
+    const int rc = run_chunk(e, tokens_host, n, e->verify_bufs, logits_out);
+    if (rc != MK_OK) return rc;
+    e->pending_verify = n;
+    return MK_OK;
+  }
   const Layout& L = e->lay;
   const size_t dn_bytes = L.conv_state[0] - L.dn_state[0];
   const size_t conv_bytes = (mk::kStateBufs > 1 ? L.dn_state[1] : L.kc) - L.conv_state[0];
@@ -805,6 +875,7 @@ int mk_debug_gemm(const void* W, const void* X, float* C, int n_out, int T, int 
   g.K = K;
   g.accumulate = 0;
   g.x_lo_row = T;
+  g.k_split = 1;
   g.err = err_word;
   g.wait_ns = 2000000000LL;
   const dim3 grid((n_out + mk::pf::BM - 1) / mk::pf::BM, (T + mk::pf::BN - 1) / mk::pf::BN);

@@ -35,6 +35,12 @@ constexpr uint32_t TILE_X_BYTES = BN * BK * 2;
 constexpr uint32_t STAGE_BYTES = TILE_W_BYTES + 2 * TILE_X_BYTES;  // W, x_hi, x_lo
 constexpr size_t GEMM_SMEM = size_t(STAGES) * STAGE_BYTES + 1024 + 256;
 
+// Per-position state copies of a verify chunk: p[t] receives the state after
+// position t (p[0] == nullptr: a prompt chunk, the state is updated in place).
+struct Ckpt {
+  float* p[kMaxVerify];
+};
+
 struct GemmArgs {
   CUtensorMap tw;    // weights [n_out][K] bf16, box {BK, BM}
   CUtensorMap tx;    // activations [2][x_lo_row][K] bf16 (hi rows, then lo rows), box {BK, BN}
@@ -42,6 +48,7 @@ struct GemmArgs {
   int ldc;
   int n_out, T, K;
   int x_lo_row;      // row of the lo half's first row in tx
+  int k_split;       // gridDim.z: K ranges summed into c with atomic adds (c pre-set by the caller)
   int accumulate;    // 1: c += result (residual add)
   int* err;
   long long wait_ns;
@@ -162,7 +169,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc(const __grid_constant
   GemmSmem* gs = reinterpret_cast<GemmSmem*>(sX + size_t(STAGES) * 2 * TILE_X_BYTES);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n0 = blockIdx.x * BM, t0 = blockIdx.y * BN;
-  const int nkb = a.K / BK;
+  // this CTA's share of the K blocks (split-K when few output tiles exist)
+  const int kb_all = a.K / BK;
+  const int kb0 = int(blockIdx.z) * kb_all / a.k_split;
+  const int nkb = (int(blockIdx.z) + 1) * kb_all / a.k_split - kb0;
 
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -188,9 +198,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc(const __grid_constant
         break;
       mbar_arrive_expect_tx(&gs->full[s], STAGE_BYTES);
       unsigned char* xs = sX + size_t(s) * 2 * TILE_X_BYTES;
-      tma_load_2d(sW + size_t(s) * TILE_W_BYTES, &a.tw, kb * BK, n0, &gs->full[s]);
-      tma_load_2d(xs, &a.tx, kb * BK, t0, &gs->full[s]);
-      tma_load_2d(xs + TILE_X_BYTES, &a.tx, kb * BK, a.x_lo_row + t0, &gs->full[s]);
+      const int kc = (kb0 + kb) * BK;
+      tma_load_2d(sW + size_t(s) * TILE_W_BYTES, &a.tw, kc, n0, &gs->full[s]);
+      tma_load_2d(xs, &a.tx, kc, t0, &gs->full[s]);
+      tma_load_2d(xs + TILE_X_BYTES, &a.tx, kc, a.x_lo_row + t0, &gs->full[s]);
       ++issued;
     }
     // copies still in flight must land before the CTA can exit
@@ -233,7 +244,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc(const __grid_constant
           const int t = t0 + c0 + i;
           if (t < a.T) {
             float* dst = a.c + size_t(t) * a.ldc + n;
-            *dst = a.accumulate ? *dst + v[i] : v[i];
+            if (a.k_split > 1) atomicAdd(dst, v[i]);
+            else *dst = a.accumulate ? *dst + v[i] : v[i];
           }
         }
       }
@@ -287,13 +299,25 @@ __global__ void rmsnorm_bf16_kernel(const float* X, const uint16_t* gain, uint16
 
 // Causal depthwise conv + SiLU over T positions, in place on the q|k|v
 // columns of P; the history (last three inputs) carries over in `state`.
+// With checkpoints the history after position t goes to ck.p[t] (same
+// [channel] float4 layout) and `state` is left as it was.
 __global__ void conv_kernel(float* P, int ldp, float4* state, const uint16_t* conv_w, int ch,
-                            int T) {
+                            int T, Ckpt ck) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= ch) return;
   float4 s = state[c];
   const uint2 wc = *reinterpret_cast<const uint2*>(conv_w + size_t(c) * 4);
   const float w0 = bf_lo(wc.x), w1 = bf_hi(wc.x), w2 = bf_lo(wc.y), w3 = bf_hi(wc.y);
+  if (ck.p[0]) {
+    for (int t = 0; t < T; ++t) {
+      const float u = P[size_t(t) * ldp + c];
+      const float y = w0 * s.x + w1 * s.y + w2 * s.z + w3 * u;
+      s = make_float4(s.y, s.z, u, 0.f);
+      P[size_t(t) * ldp + c] = siluf_(y);
+      reinterpret_cast<float4*>(ck.p[t])[c] = s;
+    }
+    return;
+  }
   int t = 0;
   for (; t + 8 <= T; t += 8) {
     float u[8];
@@ -362,7 +386,7 @@ constexpr int REC_WARPS = 8;
 template <int DK, int RPW>
 __global__ void __launch_bounds__(REC_WARPS * 32) recurrence_kernel(
     float* S, const float* QK, const float4* BAK, const float* P, int ldp, int vcol, float* O,
-    int ldo, int nh, int T) {
+    int ldo, int nh, int T, Ckpt ck) {
   constexpr int EPL = DK / 32;
   const int h = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -412,6 +436,13 @@ __global__ void __launch_bounds__(REC_WARPS * 32) recurrence_kernel(
       for (int e = 0; e < EPL; ++e) st[r][e] = fmaf(alpha, st[r][e], u * kn[e]);
       if (lane == 0) O[size_t(t) * ldo + h * DK + row0 + r] = fmaf(alpha, sq[r], u * kq);
     }
+    if (ck.p[0]) {
+#pragma unroll
+      for (int r = 0; r < RPW; ++r)
+#pragma unroll
+        for (int e = 0; e < EPL; ++e)
+          ck.p[t][(size_t(h) * DK + row0 + r) * DK + lane * EPL + e] = st[r][e];
+    }
 #pragma unroll
     for (int e = 0; e < EPL; ++e) {
       qn[e] = qn2[e];
@@ -421,6 +452,7 @@ __global__ void __launch_bounds__(REC_WARPS * 32) recurrence_kernel(
     for (int r = 0; r < RPW; ++r) vv[r] = vv2[r];
     g = g2;
   }
+  if (ck.p[0]) return;  // verify chunk: the source state stays as it was
 #pragma unroll
   for (int r = 0; r < RPW; ++r)
 #pragma unroll
@@ -476,6 +508,22 @@ __global__ void rope_kv_kernel(float* P, int ldp, int nq, int nkv, int hd, uint1
   }
 }
 
+// EPL consecutive bf16 values -> fp32 (one 4/8/16-byte load).
+template <int EPL>
+__device__ __forceinline__ void load_bf16_row(const uint16_t* p, float* f) {
+  if constexpr (EPL == 8) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    f[0] = bf_lo(u.x); f[1] = bf_hi(u.x); f[2] = bf_lo(u.y); f[3] = bf_hi(u.y);
+    f[4] = bf_lo(u.z); f[5] = bf_hi(u.z); f[6] = bf_lo(u.w); f[7] = bf_hi(u.w);
+  } else if constexpr (EPL == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    f[0] = bf_lo(u.x); f[1] = bf_hi(u.x); f[2] = bf_lo(u.y); f[3] = bf_hi(u.y);
+  } else {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+    f[0] = bf_lo(u); f[1] = bf_hi(u);
+  }
+}
+
 // Causal attention of T new positions over the cache (positions 0 ..
 // pos0+t for query t): one warp per (query, head), online softmax; the
 // output is written as split bf16 operands for the output-projection GEMM.
@@ -500,27 +548,14 @@ __global__ void attn_prefill_kernel(const float* P, int ldp, const uint16_t* kc,
 #pragma unroll
   for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
   const int nkeys = pos0 + q_idx + 1;
-  auto ld_row = [](const uint16_t* p, float* f) {
-    if constexpr (EPL == 8) {
-      const uint4 u = *reinterpret_cast<const uint4*>(p);
-      f[0] = bf_lo(u.x); f[1] = bf_hi(u.x); f[2] = bf_lo(u.y); f[3] = bf_hi(u.y);
-      f[4] = bf_lo(u.z); f[5] = bf_hi(u.z); f[6] = bf_lo(u.w); f[7] = bf_hi(u.w);
-    } else if constexpr (EPL == 4) {
-      const uint2 u = *reinterpret_cast<const uint2*>(p);
-      f[0] = bf_lo(u.x); f[1] = bf_hi(u.x); f[2] = bf_lo(u.y); f[3] = bf_hi(u.y);
-    } else {
-      const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
-      f[0] = bf_lo(u); f[1] = bf_hi(u);
-    }
-  };
   constexpr int KB = 4;  // keys in flight per step
   for (int j0 = 0; j0 < nkeys; j0 += KB) {
     float kf[KB][EPL], vf[KB][EPL], s[KB];
 #pragma unroll
     for (int u = 0; u < KB; ++u) {
       const int j = min(j0 + u, nkeys - 1);
-      ld_row(K + size_t(j) * HD + lane * EPL, kf[u]);
-      ld_row(V + size_t(j) * HD + lane * EPL, vf[u]);
+      load_bf16_row<EPL>(K + size_t(j) * HD + lane * EPL, kf[u]);
+      load_bf16_row<EPL>(V + size_t(j) * HD + lane * EPL, vf[u]);
     }
 #pragma unroll
     for (int u = 0; u < KB; ++u) {
@@ -545,6 +580,95 @@ __global__ void attn_prefill_kernel(const float* P, int ldp, const uint16_t* kc,
   uint16_t* orow = Ob + size_t(q_idx) * ldob + h * HD + lane * EPL;
 #pragma unroll
   for (int e = 0; e < EPL; ++e) store_split(orow + e, lo, acc[e] / l);
+}
+
+// Short chunks (verify): attention split over the keys as well, so a few
+// queries over a long cache still occupy the GPU.  One warp per (query t,
+// head h, key range s of ATT_SPLIT_LEN positions) writes an unnormalised
+// partial {acc[HD], m, l}; attn_merge_kernel combines the ranges.
+constexpr int ATT_SPLIT_LEN = 64;
+constexpr int ATT_SPLIT_WARPS = 4;
+
+template <int HD>
+__global__ void __launch_bounds__(ATT_SPLIT_WARPS * 32) attn_split_kernel(
+    const float* P, int ldp, const uint16_t* kc, const uint16_t* vc, int max_ctx, int nq,
+    int nkv, int pos0, int nsplit, float* part) {
+  constexpr int EPL = HD / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sidx = blockIdx.x * ATT_SPLIT_WARPS + warp;
+  const int h = blockIdx.y, t = blockIdx.z;
+  if (sidx >= nsplit) return;
+  const int g = h / (nq / nkv);
+  const int nkeys = pos0 + t + 1;
+  const int k0 = sidx * ATT_SPLIT_LEN, k1 = min(k0 + ATT_SPLIT_LEN, nkeys);
+  float* out = part + ((size_t(t) * nq + h) * nsplit + sidx) * (HD + 2);
+  float q[EPL];
+  const float* qrow = P + size_t(t) * ldp + h * HD;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) q[e] = qrow[lane * EPL + e];
+  const float scale = 1.0f / sqrtf(float(HD));
+  const uint16_t* K = kc + size_t(g) * max_ctx * HD;
+  const uint16_t* V = vc + size_t(g) * max_ctx * HD;
+  float m = -INFINITY, l = 0.f, acc[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+  constexpr int KB = 4;
+  for (int j0 = k0; j0 < k1; j0 += KB) {
+    float kf[KB][EPL], vf[KB][EPL], sc[KB];
+#pragma unroll
+    for (int u = 0; u < KB; ++u) {
+      const int j = min(j0 + u, k1 - 1);
+      load_bf16_row<EPL>(K + size_t(j) * HD + lane * EPL, kf[u]);
+      load_bf16_row<EPL>(V + size_t(j) * HD + lane * EPL, vf[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < KB; ++u) {
+      sc[u] = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) sc[u] = fmaf(q[e], kf[u][e], sc[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < KB; ++u) sc[u] = warp_sum(sc[u]) * scale;
+#pragma unroll
+    for (int u = 0; u < KB; ++u) {
+      if (j0 + u < k1) {
+        const float mn = fmaxf(m, sc[u]);
+        const float corr = expf(m - mn), p = expf(sc[u] - mn);
+        l = l * corr + p;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) acc[e] = fmaf(p, vf[u][e], acc[e] * corr);
+        m = mn;
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) out[lane * EPL + e] = acc[e];
+  if (lane == 0) {
+    out[HD] = m;  // -inf when the range holds no key of this query
+    out[HD + 1] = l;
+  }
+}
+
+// o[t][h] = sum_s e^(m_s - M) acc_s / sum_s e^(m_s - M) l_s, written as split
+// bf16 operands for the output-projection GEMM.  grid (nq, T), HD threads.
+template <int HD>
+__global__ void attn_merge_kernel(const float* part, int nq, int nsplit, uint16_t* Ob, int ldob,
+                                  size_t lo) {
+  const int h = blockIdx.x, t = blockIdx.y, i = threadIdx.x;
+  const float* base = part + (size_t(t) * nq + h) * nsplit * (HD + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, base[size_t(s) * (HD + 2) + HD]);
+  float den = 0.f, num = 0.f;
+  for (int s = 0; s < nsplit; ++s) {
+    const float* ps = base + size_t(s) * (HD + 2);
+    const float ls = ps[HD + 1];
+    if (ls > 0.f) {
+      const float wgt = expf(ps[HD] - M);
+      den = fmaf(wgt, ls, den);
+      num = fmaf(wgt, ps[i], num);
+    }
+  }
+  store_split(Ob + size_t(t) * ldob + h * HD + i, lo, num / den);
 }
 
 }  // namespace pf

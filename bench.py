@@ -38,6 +38,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extras", action="store_true",
+                   help="skip the long-context, verify, prefill-roofline and delta-sweep lines")
     p.add_argument("--mode", choices=["full", "kernel"], default="full",
                    help="kernel: W+K single decode launches at context 520 on a "
                         "seeded synthetic state (small case for profilers)")
@@ -218,6 +220,141 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+def matrix_params(cfg):
+    """Weights of every projection matrix of the layer stack (no embedding)."""
+    import numpy as np
+    from attention_decode_megakernel_b200 import synth
+    n = 0
+    for is_attn in cfg.layer_is_attn:
+        for name, shape, kind in synth.layer_tensor_shapes(cfg, is_attn):
+            if len(shape) == 2 and shape[1] > 4:  # [out][in] matrices (not conv taps)
+                n += int(np.prod(shape))
+    return n
+
+
+def state_to_device(torch, np, st):
+    return {k: (torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v).cuda()
+                if isinstance(v, np.ndarray) else v) for k, v in st.items()}
+
+
+def extra_workloads(mk, synth, torch, np, prefill_ms_per_call, hbm, tc_peak, peak_kind):
+    """The other configurations of the method, each timed on the device with
+    CUDA events: long-context decode, 5-token verify, the prompt path's
+    tensor-core roofline and the isolated delta-step sweep."""
+    out = {}
+    # prompt path: algorithmic FLOPs of pp520 (every matrix once per position,
+    # LM head for the last position only) over the measured prefill time
+    cfg = synth.hybrid_08b_config(max_ctx=PROMPT + GEN + 8)
+    flops = 2.0 * matrix_params(cfg) * PROMPT + 2.0 * cfg.vocab * cfg.hidden
+    tf = flops / (prefill_ms_per_call / 1000.0) / 1e12
+    out["prefill_pp520"] = {"tok_s": PROMPT / (prefill_ms_per_call / 1000.0),
+                            "ms": prefill_ms_per_call, "gflop": flops / 1e9,
+                            "roofline": {"bound": "tensor", "achieved": tf, "peak": tc_peak,
+                                         "unit": "TFLOP/s", "frac": tf / tc_peak,
+                                         "peak_kind": peak_kind}}
+    del cfg
+
+    # long context: the attention layers' KV at 32768 positions (synthetic
+    # state of that shape), then 32 greedy decode launches
+    ctx = 32768
+    cfg = synth.hybrid_08b_config(max_ctx=ctx + 64)
+    w = synth.make_weights(cfg)
+    eng = mk.Engine(cfg, w)
+    dev = state_to_device(torch, np, synth.make_engine_state(cfg, ctx=ctx))
+    eng.set_state(dev)
+    toks = torch.zeros(32, dtype=torch.int32, device="cuda")
+    eng.generate(1, 4, toks)
+    eng.sync()
+    eng.set_state(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(eng.stream)
+    eng.generate(1, 32, toks)
+    e1.record(eng.stream)
+    eng.sync()
+    ms = e0.elapsed_time(e1) / 32
+    byts = sum(decode_bytes(cfg, ctx + i) for i in range(32)) / 32
+    out["decode_ctx32k"] = {"tok_s": 1000.0 / ms, "ms_per_token": ms,
+                            "roofline": {"bound": "hbm", "achieved": byts / ms / 1e6,
+                                         "peak": hbm, "unit": "GB/s",
+                                         "frac": byts / ms / 1e6 / hbm,
+                                         "bytes_per_launch": byts}}
+    eng.close()
+    del eng, dev
+
+    # speculative-verify shape: context 4096, 200 calls of 5 tokens (the
+    # accepted token + 4 seeded drafts); draft j is kept while it equals the
+    # greedy choice at position j-1
+    ctx = 4096
+    cfg = synth.hybrid_08b_config(max_ctx=ctx + 256)
+    eng = mk.Engine(cfg, w)
+    eng.set_state(state_to_device(torch, np, synth.make_engine_state(cfg, ctx=ctx)))
+    drafts = synth.make_tokens(cfg.vocab, 4 * 220, seed=synth.SEED_DRAFTS).reshape(220, 4)
+    vl = torch.empty((5, cfg.vocab), dtype=torch.float32, device="cuda")
+    calls, kept, tok = 200, 0, 1
+    for i in range(calls + 5):
+        if i == 5:
+            eng.sync()
+            t0 = time.perf_counter()
+            e0.record(eng.stream)
+            kept = 0
+        seq = np.concatenate([[tok], drafts[i % 220]]).astype(np.int32)
+        eng.verify(seq, vl)
+        am = torch.argmax(vl, dim=1).cpu().numpy()
+        k = 1
+        while k < 5 and seq[k] == am[k - 1]:
+            k += 1
+        eng.accept(k)
+        kept += k
+        tok = int(am[k - 1])
+    e1.record(eng.stream)
+    eng.sync()
+    wall = time.perf_counter() - t0
+    dev_ms = e0.elapsed_time(e1)
+    weights = decode_bytes(cfg, 0) - cfg.vocab * 4 - 2 * cfg.n_attn * 2 * cfg.kv_heads * cfg.head_dim * 2
+    dn = cfg.n_dn * cfg.dn_heads * cfg.dn_dv * cfg.dn_dk * 4
+    conv = cfg.n_dn * cfg.conv_channels * (cfg.conv_k - 1) * 4
+    kvb = cfg.n_attn * 2 * cfg.kv_heads * cfg.head_dim * 2
+    vbytes = weights + dn + conv + 5 * (dn + conv) + kvb * (ctx + 100) + 5 * kvb + 5 * cfg.vocab * 4
+    out["verify_5tok_ctx4096"] = {
+        "calls_s": calls / (dev_ms / 1000.0), "ms_per_call": dev_ms / calls,
+        "positions_s": 5 * calls / (dev_ms / 1000.0), "accepted_per_call": kept / calls,
+        "wall_calls_s": calls / wall,
+        "roofline": {"bound": "hbm", "achieved": vbytes / (dev_ms / calls) / 1e6, "peak": hbm,
+                     "unit": "GB/s", "frac": vbytes / (dev_ms / calls) / 1e6 / hbm,
+                     "bytes_per_call": vbytes}}
+    eng.close()
+    del eng, w
+
+    # isolated gated delta-rule step: B sequences x 16 heads, dk = dv = 128,
+    # 1024 sequential steps, one launch per step
+    sweep = {}
+    for B in (1, 8, 64):
+        H, D, steps = 16, 128, 1024
+        S = torch.randn(B, H, D, D, device="cuda") * 0.1
+        q = torch.nn.functional.normalize(torch.randn(8, B, H, D, device="cuda"), dim=-1)
+        k = torch.nn.functional.normalize(torch.randn(8, B, H, D, device="cuda"), dim=-1)
+        q16, k16 = q.to(torch.bfloat16).view(torch.int16), k.to(torch.bfloat16).view(torch.int16)
+        v16 = torch.randn(8, B, H, D, device="cuda").to(torch.bfloat16).view(torch.int16)
+        be = torch.rand(8, B, H, device="cuda")
+        al = 0.9 + 0.1 * torch.rand(8, B, H, device="cuda")
+        o = torch.empty(B, H, D, device="cuda")
+        for t in range(16):
+            mk.mk_delta_step(S, q16[t % 8], k16[t % 8], v16[t % 8], al[t % 8], be[t % 8], o)
+        torch.cuda.synchronize()
+        e0.record()
+        for t in range(steps):
+            mk.mk_delta_step(S, q16[t % 8], k16[t % 8], v16[t % 8], al[t % 8], be[t % 8], o)
+        e1.record()
+        torch.cuda.synchronize()
+        us = 1000.0 * e0.elapsed_time(e1) / steps
+        sb = 2 * B * H * D * D * 4 + B * H * (3 * D * 2 + 8 + D * 4)
+        sweep["B%d" % B] = {"us_per_step": us, "state_GBps": sb / us / 1e3,
+                            "frac": sb / us / 1e3 / hbm, "bytes_per_step": sb}
+        del S, q, k, q16, k16, v16, be, al, o
+    out["delta_sweep_dk128_h16"] = sweep
+    return out
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -325,6 +462,12 @@ def main():
                "sample": "%d greedy decode steps of the 0.8B-shaped model at context 520 "
                          "(seeded synthetic state) in %.1f s, fp64 oracle" % (n, dt)}
 
+    extras = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        eng_ms = prefill_ms / args.steps
+        _, tc_peak, pk = peaks()
+        extras = extra_workloads(mk, synth, torch, np, eng_ms, hbm, tc_peak, pk)
+
     line = {
         "metric": "batch-1 decode tok/s (tg128)", "value": value, "unit": "tok/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -346,6 +489,7 @@ def main():
         "clocks": clocks,
         "cpu_baseline": cpu,
         "greedy_tokens_head": out_tokens[:8],
+        "extras": extras,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

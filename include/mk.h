@@ -151,10 +151,17 @@ int mk_decode_step(mk_engine *e, int32_t token, float *logits_out);
 int mk_generate(mk_engine *e, int32_t first_token, int n, int32_t *tokens_out,
                 float *logits_out);
 
-/* Verify n tokens at once (1 <= n <= max_verify): the stack runs over
- * positions pos .. pos+n-1 exactly as n decode steps would, writing the logits of every position to logits_out (device, float32
- * [n][vocab], not NULL) and a checkpoint of the recurrent state after each
- * position.  The position does not advance until mk_accept. */
+/* Verify n tokens at once (1 <= n <= max_verify), the speculative-decoding
+ * shape (several draft tokens checked by one forward pass, with the
+ * recurrent state checkpointed for rollback): the stack runs over positions
+ * pos .. pos+n-1 as one chunk -- every projection one tensor-core GEMM with
+ * M = n (weights read once for the n positions), the conv and the gated
+ * delta rule advanced position by position -- and writes the logits of
+ * every position to logits_out (device, float32 [n][vocab], not NULL), the
+ * DeltaNet and conv state after each position to its own checkpoint buffer,
+ * and K/V of the n positions to the cache.  Results equal n decode steps up
+ * to rounding.  The current state is left as it was; the position does not
+ * advance until mk_accept.  MK_ERR_STATE while a verify is pending. */
 int mk_verify(mk_engine *e, const int32_t *tokens_host, int n,
               float *logits_out);
 

@@ -236,8 +236,8 @@ class OracleModel:
 
     def __del__(self):
         h = getattr(self, "_h", None)
-        if h:
-            lib().orc_destroy(h)
+        if h and _lib is not None:  # not during interpreter shutdown
+            _lib.orc_destroy(h)
             self._h = None
 
     def clone(self) -> "OracleModel":

@@ -178,33 +178,73 @@ def test_generate_equals_decode_loop_bitwise(mk):
     assert torch.equal(sa, sb)
 
 
-def test_verify_then_accept_equals_sequential_decode(mk):
+@pytest.mark.parametrize("cfg_name,keep", [("tiny", 1), ("tiny", 3), ("tiny", 5), ("mid", 2)])
+def test_verify_against_oracle_then_accept(mk, cfg_name, keep):
+    """Speculative-verify shape: 5 tokens (1 accepted + 4 drafts) in one
+    call.  Every position's logits must match the oracle stepping the same
+    tokens; the current state must be untouched until mk_accept; after
+    accepting `keep` positions the state equals the oracle's after those
+    positions and decoding continues from it."""
+    cfg = (synth.tiny_config(max_ctx=256) if cfg_name == "tiny"
+           else synth.hybrid_mid_config(max_ctx=256))
+    w = synth.make_weights(cfg)
+    prompt = synth.make_tokens(cfg.vocab, 40)
+    drafts = synth.make_tokens(cfg.vocab, 5, seed=synth.SEED_DRAFTS)
+    eng = mk.Engine(cfg, w)
+    orc = oracle.OracleModel(cfg, w)
+    eng.prefill(prompt)
+    for t in prompt:
+        orc.step(int(t))
+    before = [x.clone() for x in eng.get_state()[:2]]
+    vl = torch.empty((5, cfg.vocab), dtype=torch.float32, device="cuda")
+    eng.verify(drafts, vl)
+    eng.sync()
+    assert eng.position == 40
+    after = eng.get_state()[:2]
+    assert torch.equal(before[0], after[0]) and torch.equal(before[1], after[1])
+    tr = Tracker()
+    ref_orc = orc.clone()
+    for j in range(5):
+        ref, _ = ref_orc.step(int(drafts[j]))
+        tr.logits(_np(vl[j]), ref)
+    eng.accept(keep)
+    assert eng.position == 40 + keep
+    for j in range(keep):
+        ref, _ = orc.step(int(drafts[j]))
+    _check_state(eng, orc)
+    _teacher_forced(eng, orc, cfg, int(np.argmax(ref)), 3, tr)
+    print(tr.finish())
+
+
+def test_verify_twice_and_cycle_buffers(mk):
+    """Repeated verify/accept cycles walk the checkpoint buffers round the
+    ring; the result tracks the oracle."""
     cfg = synth.tiny_config(max_ctx=256)
     w = synth.make_weights(cfg)
-    prompt = synth.make_tokens(cfg.vocab, 12)
-    drafts = synth.make_tokens(cfg.vocab, 5, seed=synth.SEED_DRAFTS)
-    a, b = mk.Engine(cfg, w), mk.Engine(cfg, w)
-    a.prefill(prompt)
-    b.prefill(prompt)
-    vl = torch.empty((5, cfg.vocab), dtype=torch.float32, device="cuda")
-    a.verify(drafts, vl)
-    assert a.position == 12
-    dl = torch.empty((5, cfg.vocab), dtype=torch.float32, device="cuda")
-    for j in range(5):
-        b.decode_step(int(drafts[j]), dl[j])
-    assert torch.equal(vl, dl)
-    # keep 2: state equals a fresh engine that decoded exactly 2 drafts
-    a.accept(2)
-    assert a.position == 14
-    c = mk.Engine(cfg, w)
-    c.prefill(prompt)
-    c.prefill(drafts[:2])
-    assert torch.equal(a.get_state()[0], c.get_state()[0])
-    assert torch.equal(a.get_state()[1], c.get_state()[1])
-    la, lc = torch.empty_like(dl[0]), torch.empty_like(dl[0])
-    a.decode_step(7, la)
-    c.decode_step(7, lc)
-    assert torch.equal(la, lc)
+    eng = mk.Engine(cfg, w)
+    orc = oracle.OracleModel(cfg, w)
+    prompt = synth.make_tokens(cfg.vocab, 16)
+    eng.prefill(prompt)
+    for t in prompt:
+        orc.step(int(t))
+    rng = np.random.default_rng(11)
+    tr = Tracker()
+    vl = torch.empty((8, cfg.vocab), dtype=torch.float32, device="cuda")
+    for it in range(6):
+        n = int(rng.integers(1, 9))
+        toks = rng.integers(0, cfg.vocab, n)
+        eng.verify(toks, vl[:n])
+        eng.sync()
+        keep = int(rng.integers(1, n + 1))
+        ref_orc = orc.clone()
+        for j in range(n):
+            ref, _ = ref_orc.step(int(toks[j]))
+            tr.logits(_np(vl[j]), ref)
+        eng.accept(keep)
+        for j in range(keep):
+            orc.step(int(toks[j]))
+    _check_state(eng, orc)
+    print(tr.finish())
 
 
 def test_engine_errors(mk):
