@@ -406,24 +406,6 @@ __device__ __forceinline__ void dot4(const unsigned char* r0, const unsigned cha
   for (int q = 0; q < 4; ++q) acc[q] = s[q][0] + s[q][1];
 }
 
-// Warp reduction of four values at once (6 shuffles instead of 20): on
-// return lanes 8q .. 8q+7 hold the warp-wide sum of input q.
-__device__ __forceinline__ float reduce4(float a, float b, float c, float d, int lane) {
-  const bool h16 = (lane & 16) != 0;
-  float x0 = h16 ? c : a, x1 = h16 ? d : b;
-  const float y0 = h16 ? a : c, y1 = h16 ? b : d;
-  x0 += __shfl_xor_sync(0xffffffffu, y0, 16);
-  x1 += __shfl_xor_sync(0xffffffffu, y1, 16);
-  const bool h8 = (lane & 8) != 0;
-  float z = h8 ? x1 : x0;
-  const float w = h8 ? x0 : x1;
-  z += __shfl_xor_sync(0xffffffffu, w, 8);
-  z += __shfl_xor_sync(0xffffffffu, z, 4);
-  z += __shfl_xor_sync(0xffffffffu, z, 2);
-  z += __shfl_xor_sync(0xffffffffu, z, 1);
-  return z;
-}
-
 // ---- matrix phases ------------------------------------------------------------
 // One routine serves every matrix phase, so the hot loop exists once in the
 // instruction stream (a phase switch then finds it cached); the epilogue is a

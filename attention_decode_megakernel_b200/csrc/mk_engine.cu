@@ -26,7 +26,7 @@ struct Layout {
   size_t x, inp, dno, qkv, atto, mlph, part, hidden, logits, tickets, err, amax;
   // multi-token prompt path: T_MAX positions per chunk
   int tmax, pw, aw;
-  size_t pf_tok, pf_x, pf_xn, pf_p, pf_o, pf_a16, pf_qk, pf_bak, pf_att;
+  size_t pf_tok, pf_x, pf_xn, pf_p, pf_c, pf_o, pf_a16, pf_qk, pf_bak, pf_att;
   size_t total;
 };
 
@@ -99,6 +99,7 @@ Layout make_layout(const mk_config& c) {
     L.pf_x = take(size_t(T) * c.hidden * 4);
     L.pf_xn = take(size_t(2) * T * c.hidden * 2);  // [hi|lo][T][H] bf16
     L.pf_p = take(size_t(T) * pw * 4);
+    L.pf_c = take(size_t(T) * ch * 4);  // conv output of the q|k|v channels
     L.pf_o = take(size_t(T) * c.dn_heads * c.dn_dv * 4);
     L.pf_a16 = take(size_t(2) * T * aw * 2);  // [hi|lo][T][aw] bf16
     L.pf_qk = take(size_t(c.dn_heads) * T * 2 * c.dn_dk * 4);
@@ -326,19 +327,31 @@ int run_chunk(mk_engine* e, const int32_t* tokens_host, int T, const int* ck_buf
           ckc.p[t] = m.conv_state[ck_bufs[t]] + size_t(D.sub) * m.ch * 4;
           cks.p[t] = m.dn_state[ck_bufs[t]] + size_t(D.sub) * nh * dv * dk;
         }
-      conv_kernel<<<(m.ch + 255) / 256, 256, 0, st>>>(
-          P, pw, reinterpret_cast<float4*>(m.conv_state[e->cur_buf]) + size_t(D.sub) * m.ch,
-          D.conv_w, m.ch, T, ckc);
-      dn_prep_kernel<<<dim3(T, nh), dk, 0, st>>>(P, pw, nh, dk, m.ch, dv, D.A_log, D.dt_bias, QK,
-                                                 BAK, T);
+      float4* cst = reinterpret_cast<float4*>(m.conv_state[e->cur_buf]) + size_t(D.sub) * m.ch;
+      float* Cv = reinterpret_cast<float*>(ws + L.pf_c);
+      conv_kernel<<<dim3((m.ch + 255) / 256, T), 256, 0, st>>>(P, pw, cst, D.conv_w, m.ch, Cv,
+                                                              m.ch, ckc);
+      if (!ck_bufs) {
+        conv_state_kernel<<<(m.ch + 255) / 256, 256, 0, st>>>(P, pw, cst, m.ch, T);
+        e->launches += 1;
+      }
+      dn_prep_kernel<<<dim3(T, nh), dk, 0, st>>>(Cv, m.ch, P, pw, nh, dk, m.ch, dv, D.A_log,
+                                                 D.dt_bias, QK, BAK, T);
       float* S = m.dn_state[e->cur_buf] + size_t(D.sub) * nh * dv * dk;
-      const dim3 rgrid(nh, dv / (REC_WARPS * 2));
-      if (dk == 128)
-        recurrence_kernel<128, 2><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, P, pw, 2 * nh * dk,
-                                                                    O, nh * dv, nh, T, cks);
+      const dim3 rgrid(nh, dv / (REC_WARPS * REC_RPW));
+      const int vcol = 2 * nh * dk;
+      if (dk == 128 && ck_bufs)
+        recurrence_kernel<128, true><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, Cv, m.ch, vcol,
+                                                                       O, nh * dv, T, cks);
+      else if (dk == 128)
+        recurrence_kernel<128, false><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, Cv, m.ch, vcol,
+                                                                        O, nh * dv, T, cks);
+      else if (ck_bufs)
+        recurrence_kernel<64, true><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, Cv, m.ch, vcol,
+                                                                      O, nh * dv, T, cks);
       else
-        recurrence_kernel<64, 2><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, P, pw, 2 * nh * dk,
-                                                                   O, nh * dv, nh, T, cks);
+        recurrence_kernel<64, false><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, Cv, m.ch, vcol,
+                                                                       O, nh * dv, T, cks);
       gated_norm_kernel<<<dim3(T, nh), dv, 0, st>>>(O, nh * dv, P, pw, m.ch, D.out_norm, A16, aw,
                                                     c.rms_eps, lo_a);
       if (rc == MK_OK) rc = launch_gemm(e, mp.out, e->map_a16_dn, X, H, H, T, nh * dv, 1);

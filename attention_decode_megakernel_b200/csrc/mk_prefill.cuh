@@ -297,58 +297,50 @@ __global__ void rmsnorm_bf16_kernel(const float* X, const uint16_t* gain, uint16
     store_split(Xn + size_t(t) * H + i, lo, x[i] * inv * bf2f(gain[i]));
 }
 
-// Causal depthwise conv + SiLU over T positions, in place on the q|k|v
-// columns of P; the history (last three inputs) carries over in `state`.
-// With checkpoints the history after position t goes to ck.p[t] (same
-// [channel] float4 layout) and `state` is left as it was.
-__global__ void conv_kernel(float* P, int ldp, float4* state, const uint16_t* conv_w, int ch,
-                            int T, Ckpt ck) {
+// Causal depthwise conv + SiLU over T positions, one thread per (position,
+// channel): Cv[t][c] = SiLU(w0 u_{t-3} + w1 u_{t-2} + w2 u_{t-1} + w3 u_t)
+// with u = the raw in-projection columns of P and u_{<0} taken from the
+// carried history `state` = (u_{-3}, u_{-2}, u_{-1}).  With checkpoints the
+// history after position t, (u_{t-2}, u_{t-1}, u_t), goes to ck.p[t].
+__device__ __forceinline__ float conv_input(const float* P, int ldp, const float4& s, int t,
+                                            int c) {
+  return t >= 0 ? P[size_t(t) * ldp + c] : (t == -1 ? s.z : t == -2 ? s.y : s.x);
+}
+
+__global__ void conv_kernel(const float* P, int ldp, const float4* state, const uint16_t* conv_w,
+                            int ch, float* Cv, int ldc, Ckpt ck) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x, t = blockIdx.y;
+  if (c >= ch) return;
+  const float4 s = state[c];
+  const uint2 wc = *reinterpret_cast<const uint2*>(conv_w + size_t(c) * 4);
+  const float u3 = conv_input(P, ldp, s, t - 3, c), u2 = conv_input(P, ldp, s, t - 2, c);
+  const float u1 = conv_input(P, ldp, s, t - 1, c), u0 = P[size_t(t) * ldp + c];
+  const float y = bf_lo(wc.x) * u3 + bf_hi(wc.x) * u2 + bf_lo(wc.y) * u1 + bf_hi(wc.y) * u0;
+  Cv[size_t(t) * ldc + c] = siluf_(y);
+  if (ck.p[0]) reinterpret_cast<float4*>(ck.p[t])[c] = make_float4(u2, u1, u0, 0.f);
+}
+
+// The carried history after T positions (a separate launch: every conv
+// thread must have read the old one first).
+__global__ void conv_state_kernel(const float* P, int ldp, float4* state, int ch, int T) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= ch) return;
-  float4 s = state[c];
-  const uint2 wc = *reinterpret_cast<const uint2*>(conv_w + size_t(c) * 4);
-  const float w0 = bf_lo(wc.x), w1 = bf_hi(wc.x), w2 = bf_lo(wc.y), w3 = bf_hi(wc.y);
-  if (ck.p[0]) {
-    for (int t = 0; t < T; ++t) {
-      const float u = P[size_t(t) * ldp + c];
-      const float y = w0 * s.x + w1 * s.y + w2 * s.z + w3 * u;
-      s = make_float4(s.y, s.z, u, 0.f);
-      P[size_t(t) * ldp + c] = siluf_(y);
-      reinterpret_cast<float4*>(ck.p[t])[c] = s;
-    }
-    return;
-  }
-  int t = 0;
-  for (; t + 8 <= T; t += 8) {
-    float u[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) u[j] = P[size_t(t + j) * ldp + c];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float y = w0 * s.x + w1 * s.y + w2 * s.z + w3 * u[j];
-      s = make_float4(s.y, s.z, u[j], 0.f);
-      P[size_t(t + j) * ldp + c] = siluf_(y);
-    }
-  }
-  for (; t < T; ++t) {
-    const float u = P[size_t(t) * ldp + c];
-    const float y = w0 * s.x + w1 * s.y + w2 * s.z + w3 * u;
-    s = make_float4(s.y, s.z, u, 0.f);
-    P[size_t(t) * ldp + c] = siluf_(y);
-  }
-  state[c] = s;
+  const float4 s = state[c];
+  state[c] = make_float4(conv_input(P, ldp, s, T - 3, c), conv_input(P, ldp, s, T - 2, c),
+                         conv_input(P, ldp, s, T - 1, c), 0.f);
 }
 
 // Per (position, head): L2-normalised q (scaled by dk^-1/2) and k, the gates
 // beta = sigmoid(b) and alpha = exp(-exp(A_log) softplus(a + dt_bias)), and
 // k.q.  QK [nh][T][2*dk], BAK [nh][T][4] = {beta, alpha, k.q, 0}.
-__global__ void dn_prep_kernel(const float* P, int ldp, int nh, int dk, int ch, int dv,
-                               const float* A_log, const float* dt_bias, float* QK, float4* BAK,
-                               int T) {
+__global__ void dn_prep_kernel(const float* Cv, int ldc, const float* P, int ldp, int nh, int dk,
+                               int ch, int dv, const float* A_log, const float* dt_bias,
+                               float* QK, float4* BAK, int T) {
   __shared__ float red[32];
   const int t = blockIdx.x, h = blockIdx.y, i = threadIdx.x;  // blockDim.x == dk
   const float* prow = P + size_t(t) * ldp;
-  const float q = prow[h * dk + i], k = prow[nh * dk + h * dk + i];
+  const float* crow = Cv + size_t(t) * ldc;
+  const float q = crow[h * dk + i], k = crow[nh * dk + h * dk + i];
   const float sq = block_sum(q * q, red);
   const float sk = block_sum(k * k, red);
   const float qn = q / sqrtf(sq + 1e-6f) / sqrtf(float(dk));
@@ -364,100 +356,93 @@ __global__ void dn_prep_kernel(const float* P, int ldp, int nh, int dk, int ch, 
   }
 }
 
-template <int DK, int RPW>
-__device__ __forceinline__ void rec_load(const float* qk, const float4* bak, const float* P,
-                                         int ldp, int vcol, int t, int lane, float (&q)[DK / 32],
-                                         float (&k)[DK / 32], float (&v)[RPW], float4& gg) {
-  constexpr int EPL = DK / 32;
-#pragma unroll
-  for (int e = 0; e < EPL; ++e) {
-    q[e] = qk[size_t(t) * 2 * DK + lane * EPL + e];
-    k[e] = qk[size_t(t) * 2 * DK + DK + lane * EPL + e];
-  }
-#pragma unroll
-  for (int r = 0; r < RPW; ++r) v[r] = P[size_t(t) * ldp + vcol + r];
-  gg = bak[t];
-}
-
-// Gated delta rule over T positions for RPW rows per warp: the state rows
-// stay in registers; each lane holds DK/32 entries of a row.
+// Gated delta rule over T positions, the state rows in registers: each
+// warp owns RPW = 2 rows of one head (lane: DK/32 entries of a row), a block
+// 8 warps = 16 rows.  The block stages REC_TT positions of q, k, gates and
+// its v values in shared memory, then steps through them:
 //   u = beta (v - alpha S.k),  S <- alpha S + u k^T,  o = S.q = alpha S_old.q + u (k.q)
+// The four dot products of a step (S.k and S.q of both rows) share one
+// shuffle tree.  CKPT: the state after position t goes to ck.p[t] and S is
+// left as it was (verify); otherwise S is updated in place.
 constexpr int REC_WARPS = 8;
-template <int DK, int RPW>
+constexpr int REC_RPW = 2;
+constexpr int REC_TT = 32;
+template <int DK, bool CKPT>
 __global__ void __launch_bounds__(REC_WARPS * 32) recurrence_kernel(
-    float* S, const float* QK, const float4* BAK, const float* P, int ldp, int vcol, float* O,
-    int ldo, int nh, int T, Ckpt ck) {
+    float* S, const float* QK, const float4* BAK, const float* Cv, int ldc, int vcol, float* O,
+    int ldo, int T, Ckpt ck) {
   constexpr int EPL = DK / 32;
+  constexpr int BR = REC_WARPS * REC_RPW;  // rows per block
+  __shared__ __align__(16) float sqk[REC_TT][2 * DK];
+  __shared__ float4 sgate[REC_TT];
+  __shared__ float sv[REC_TT][BR];
   const int h = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row0 = (blockIdx.y * REC_WARPS + warp) * RPW;  // value coordinate i of the head
-  float st[RPW][EPL];
+  const int brow0 = blockIdx.y * BR;          // first row of the block within the head
+  const int row0 = brow0 + warp * REC_RPW;    // value coordinate i of this warp's first row
+  float st[REC_RPW][EPL];
 #pragma unroll
-  for (int r = 0; r < RPW; ++r)
+  for (int r = 0; r < REC_RPW; ++r)
 #pragma unroll
     for (int e = 0; e < EPL; ++e)
       st[r][e] = S[(size_t(h) * DK + row0 + r) * DK + lane * EPL + e];
   const float* qk = QK + size_t(h) * T * 2 * DK;
   const float4* bak = BAK + size_t(h) * T;
-  const int vc = vcol + h * DK + row0;  // v of this warp's rows
-  // one step of lookahead for the loads
-  float qn[EPL], kn[EPL], vv[RPW];
-  float4 g = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (T > 0) rec_load<DK, RPW>(qk, bak, P, ldp, vc, 0, lane, qn, kn, vv, g);
-  for (int t = 0; t < T; ++t) {
-    float qn2[EPL], kn2[EPL], vv2[RPW];
-    float4 g2 = g;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) { qn2[e] = qn[e]; kn2[e] = kn[e]; }
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) vv2[r] = vv[r];
-    if (t + 1 < T) rec_load<DK, RPW>(qk, bak, P, ldp, vc, t + 1, lane, qn2, kn2, vv2, g2);
-    float sk[RPW], sq[RPW];
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      sk[r] = 0.f;
-      sq[r] = 0.f;
+  const float* vsrc = Cv + vcol + h * DK + brow0;
+  for (int t0 = 0; t0 < T; t0 += REC_TT) {
+    const int nt = min(REC_TT, T - t0);
+    __syncthreads();  // the previous tile is consumed
+    const float4* src4 = reinterpret_cast<const float4*>(qk + size_t(t0) * 2 * DK);
+    for (int i = threadIdx.x; i < nt * (2 * DK / 4); i += blockDim.x)
+      reinterpret_cast<float4*>(&sqk[0][0])[i] = src4[i];
+    for (int i = threadIdx.x; i < nt; i += blockDim.x) sgate[i] = bak[t0 + i];
+    for (int i = threadIdx.x; i < nt * BR; i += blockDim.x)
+      sv[i / BR][i % BR] = vsrc[size_t(t0 + i / BR) * ldc + (i % BR)];
+    __syncthreads();
+    for (int tt = 0; tt < nt; ++tt) {
+      float q[EPL], k[EPL];
 #pragma unroll
       for (int e = 0; e < EPL; ++e) {
-        sk[r] = fmaf(st[r][e], kn[e], sk[r]);
-        sq[r] = fmaf(st[r][e], qn[e], sq[r]);
+        q[e] = sqk[tt][lane * EPL + e];
+        k[e] = sqk[tt][DK + lane * EPL + e];
+      }
+      const float4 g = sgate[tt];  // {beta, alpha, k.q, -}
+      float pk0 = 0.f, pq0 = 0.f, pk1 = 0.f, pq1 = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        pk0 = fmaf(st[0][e], k[e], pk0);
+        pq0 = fmaf(st[0][e], q[e], pq0);
+        pk1 = fmaf(st[1][e], k[e], pk1);
+        pq1 = fmaf(st[1][e], q[e], pq1);
+      }
+      // lanes 0-7: S0.k, 8-15: S0.q, 16-23: S1.k, 24-31: S1.q
+      const float z = reduce4(pk0, pq0, pk1, pq1, lane);
+      const float sk0 = __shfl_sync(0xffffffffu, z, 0), sk1 = __shfl_sync(0xffffffffu, z, 16);
+      const float u0 = g.x * (sv[tt][warp * REC_RPW] - g.y * sk0);
+      const float u1 = g.x * (sv[tt][warp * REC_RPW + 1] - g.y * sk1);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        st[0][e] = fmaf(g.y, st[0][e], u0 * k[e]);
+        st[1][e] = fmaf(g.y, st[1][e], u1 * k[e]);
+      }
+      if (lane == 8) O[size_t(t0 + tt) * ldo + h * DK + row0] = fmaf(g.y, z, u0 * g.z);
+      if (lane == 24) O[size_t(t0 + tt) * ldo + h * DK + row0 + 1] = fmaf(g.y, z, u1 * g.z);
+      if constexpr (CKPT) {
+#pragma unroll
+        for (int r = 0; r < REC_RPW; ++r)
+#pragma unroll
+          for (int e = 0; e < EPL; ++e)
+            ck.p[t0 + tt][(size_t(h) * DK + row0 + r) * DK + lane * EPL + e] = st[r][e];
       }
     }
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      sk[r] = warp_sum(sk[r]);
-      sq[r] = warp_sum(sq[r]);
-    }
-    const float beta = g.x, alpha = g.y, kq = g.z;
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      const float u = beta * (vv[r] - alpha * sk[r]);
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) st[r][e] = fmaf(alpha, st[r][e], u * kn[e]);
-      if (lane == 0) O[size_t(t) * ldo + h * DK + row0 + r] = fmaf(alpha, sq[r], u * kq);
-    }
-    if (ck.p[0]) {
-#pragma unroll
-      for (int r = 0; r < RPW; ++r)
-#pragma unroll
-        for (int e = 0; e < EPL; ++e)
-          ck.p[t][(size_t(h) * DK + row0 + r) * DK + lane * EPL + e] = st[r][e];
-    }
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      qn[e] = qn2[e];
-      kn[e] = kn2[e];
-    }
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) vv[r] = vv2[r];
-    g = g2;
   }
-  if (ck.p[0]) return;  // verify chunk: the source state stays as it was
+  if constexpr (!CKPT) {
 #pragma unroll
-  for (int r = 0; r < RPW; ++r)
+    for (int r = 0; r < REC_RPW; ++r)
 #pragma unroll
-    for (int e = 0; e < EPL; ++e)
-      S[(size_t(h) * DK + row0 + r) * DK + lane * EPL + e] = st[r][e];
+      for (int e = 0; e < EPL; ++e)
+        S[(size_t(h) * DK + row0 + r) * DK + lane * EPL + e] = st[r][e];
+  }
 }
 
 // G[t][h*dv + i] = split(RMSNorm_dv(O[t][h]) * w_i * SiLU(z[t][h*dv+i]))

@@ -134,6 +134,24 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// Warp reduction of four values at once (6 shuffles instead of 4 x 5): on
+// return lanes 8q .. 8q+7 hold the warp-wide sum of input q.
+__device__ __forceinline__ float reduce4(float a, float b, float c, float d, int lane) {
+  const bool h16 = (lane & 16) != 0;
+  float x0 = h16 ? c : a, x1 = h16 ? d : b;
+  const float y0 = h16 ? a : c, y1 = h16 ? b : d;
+  x0 += __shfl_xor_sync(0xffffffffu, y0, 16);
+  x1 += __shfl_xor_sync(0xffffffffu, y1, 16);
+  const bool h8 = (lane & 8) != 0;
+  float z = h8 ? x1 : x0;
+  const float w = h8 ? x0 : x1;
+  z += __shfl_xor_sync(0xffffffffu, w, 8);
+  z += __shfl_xor_sync(0xffffffffu, z, 4);
+  z += __shfl_xor_sync(0xffffffffu, z, 2);
+  z += __shfl_xor_sync(0xffffffffu, z, 1);
+  return z;
+}
+
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
 __device__ __forceinline__ float siluf_(float x) { return x / (1.0f + expf(-x)); }
 __device__ __forceinline__ float softplusf_(float x) { return x > 20.f ? x : log1pf(expf(x)); }
