@@ -88,6 +88,7 @@ def lib():
             "mk_delta_step": (C.c_int, [vp, vp, vp, vp, vp, vp, vp, C.c_int, C.c_int,
                                         C.c_int, C.c_int, vp]),
             "mk_debug_gemm": (C.c_int, [vp, vp, vp, C.c_int, C.c_int, C.c_int, vp]),
+            "mk_debug_gemm_noalloc": (C.c_int, [vp, vp, vp, C.c_int, C.c_int, C.c_int, vp]),
             "mk_strerror": (C.c_char_p, [C.c_int]),
         }
         for name, (res, args) in sig.items():
@@ -282,3 +283,16 @@ def mk_debug_gemm(W, X, Cout, stream=None):
     st = stream if stream is not None else 0
     _check(lib().mk_debug_gemm(_ptr(W), _ptr(X), _ptr(Cout), int(n_out), int(T), int(K), st),
            "mk_debug_gemm")
+
+
+def mk_debug_gemm_noalloc(W, X, Cout, stream=None):
+    """mk_debug_gemm through the allocation-free entry point (static scratch)."""
+    n_out, K = W.shape
+    if X.numel() % (2 * K):
+        raise ValueError("X must hold [2][T][K] bf16 (hi then lo operands)")
+    T = X.numel() // (2 * K)
+    if Cout.numel() != T * n_out:
+        raise ValueError("C must hold [T][n_out] float32")
+    st = stream if stream is not None else 0
+    _check(lib().mk_debug_gemm_noalloc(_ptr(W), _ptr(X), _ptr(Cout), int(n_out), int(T), int(K),
+                                       st), "mk_debug_gemm_noalloc")

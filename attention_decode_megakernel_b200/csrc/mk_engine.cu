@@ -897,6 +897,79 @@ int mk_debug_gemm(const void* W, const void* X, float* C, int n_out, int T, int 
   return cuda_status(cudaGetLastError());
 }
 
+}  // extern "C"
+
+namespace {
+// Static device scratch of the allocation-free GEMM entry point: split-K
+// partial sums (at most kNoAllocFloats floats = 8 MiB) and its wait-error
+// word (zero when the module loads; written only when a wait runs out).
+constexpr size_t kNoAllocFloats = size_t(2) << 20;
+__device__ __align__(256) float g_noalloc_partial[kNoAllocFloats];
+__device__ __align__(256) int g_noalloc_err;
+constexpr int kNoAllocMaxDevices = 64;
+float* g_partial_addr[kNoAllocMaxDevices];
+int* g_err_addr[kNoAllocMaxDevices];
+}  // namespace
+
+extern "C" {
+
+int mk_debug_gemm_noalloc(const void* W, const void* X, float* C, int n_out, int T, int K,
+                          void* stream) {
+  if (!W || !X || !C || n_out <= 0 || T <= 0 || K <= 0 || K % 64) return MK_ERR_ARG;
+  if (size_t(T) * size_t(n_out) > kNoAllocFloats) return MK_ERR_ARG;  // exceeds the static scratch
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) {
+    cudaGetLastError();
+    return MK_ERR_CUDA;
+  }
+  if (!g_partial_addr[dev]) {
+    // first call on this device (the device is current): look up the scratch
+    void* pp = nullptr;
+    void* pe = nullptr;
+    if (cudaGetSymbolAddress(&pp, g_noalloc_partial) != cudaSuccess ||
+        cudaGetSymbolAddress(&pe, g_noalloc_err) != cudaSuccess) {
+      cudaGetLastError();
+      return MK_ERR_CUDA;
+    }
+    g_err_addr[dev] = static_cast<int*>(pe);
+    g_partial_addr[dev] = static_cast<float*>(pp);
+  }
+  mk::pf::GemmArgs g;
+  if (!make_map(&g.tw, W, n_out, K, K, mk::pf::BM) ||
+      !make_map(&g.tx, X, 2 * T, K, K, mk::pf::BN))
+    return MK_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(mk::pf::gemm_tc_partial, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(mk::pf::GEMM_SMEM)) != cudaSuccess) {
+    cudaGetLastError();
+    return MK_ERR_CUDA;
+  }
+  int sms = 148;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 148;
+  const int tiles = ((n_out + mk::pf::BM - 1) / mk::pf::BM) * ((T + mk::pf::BN - 1) / mk::pf::BN);
+  int ks = (sms + tiles - 1) / tiles;
+  if (ks > K / mk::pf::BK) ks = K / mk::pf::BK;
+  while (ks > 1 && size_t(ks) * T * n_out > kNoAllocFloats) --ks;
+  if (ks < 1) ks = 1;
+  g.c = C;
+  g.ldc = n_out;
+  g.n_out = n_out;
+  g.T = T;
+  g.K = K;
+  g.accumulate = 0;
+  g.x_lo_row = T;
+  g.k_split = ks;
+  g.err = g_err_addr[dev];
+  g.wait_ns = 2000000000LL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dim3 grid((n_out + mk::pf::BM - 1) / mk::pf::BM, (T + mk::pf::BN - 1) / mk::pf::BN, ks);
+  mk::pf::gemm_tc_partial<<<grid, mk::pf::GEMM_THREADS, mk::pf::GEMM_SMEM, st>>>(
+      g, g_partial_addr[dev]);
+  const size_t n = size_t(T) * n_out;
+  const int rblocks = int((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  mk::pf::splitk_reduce_kernel<<<rblocks, 256, 0, st>>>(g_partial_addr[dev], ks, n, C);
+  return cuda_status(cudaGetLastError());
+}
+
 const char* mk_strerror(int s) {
   switch (s) {
     case MK_OK: return "ok";

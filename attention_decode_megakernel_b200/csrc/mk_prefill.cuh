@@ -160,7 +160,10 @@ __device__ __forceinline__ bool gemm_wait(uint64_t* bar, uint32_t parity, GemmSm
 }
 
 // C[t][n] (+)= sum_k X[t][k] * W[n][k] for one 128 x 128 (rows x tokens) tile.
-__global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc(const __grid_constant__ GemmArgs a) {
+// PARTIAL: K range blockIdx.z stores its sum to partial[z][T][n_out] (summed
+// afterwards in a fixed order) instead of writing c.
+template <bool PARTIAL>
+__device__ __forceinline__ void gemm_tile(const GemmArgs& a, float* partial) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -244,7 +247,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc(const __grid_constant
           const int t = t0 + c0 + i;
           if (t < a.T) {
             float* dst = a.c + size_t(t) * a.ldc + n;
-            if (a.k_split > 1) atomicAdd(dst, v[i]);
+            if constexpr (PARTIAL) partial[(size_t(blockIdx.z) * a.T + t) * a.n_out + n] = v[i];
+            else if (a.k_split > 1) atomicAdd(dst, v[i]);
             else *dst = a.accumulate ? *dst + v[i] : v[i];
           }
         }
@@ -254,6 +258,26 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc(const __grid_constant
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, BN);
+}
+
+__global__ void __launch_bounds__(GEMM_THREADS, 1) gemm_tc(const __grid_constant__ GemmArgs a) {
+  gemm_tile<false>(a, nullptr);
+}
+
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_tc_partial(const __grid_constant__ GemmArgs a, float* partial) {
+  gemm_tile<true>(a, partial);
+}
+
+// C[t][n] = sum over z of partial[z][t][n], in order z = 0, 1, ... (a split-K
+// result that does not depend on the order the ranges finished in).
+__global__ void splitk_reduce_kernel(const float* partial, int k_split, size_t n, float* c) {
+  for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += size_t(gridDim.x) * blockDim.x) {
+    float acc = 0.f;
+    for (int z = 0; z < k_split; ++z) acc += partial[size_t(z) * n + i];
+    c[i] = acc;
+  }
 }
 
 // ---- elementwise / row kernels --------------------------------------------------

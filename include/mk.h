@@ -237,6 +237,23 @@ int mk_delta_step(float *S, const void *q, const void *k, const void *v,
 int mk_debug_gemm(const void *W, const void *X, float *C, int n_out, int T,
                   int K, void *stream);
 
+/* The same GEMM as mk_debug_gemm, for callers that must not allocate device
+ * memory (the pages have no counterpart): a process whose device memory is
+ * fully budgeted up front, or a host loop that may not call cudaMalloc or an
+ * allocating library between steps.  It allocates nothing: K is split over
+ * the SMs and the ranges' partial sums go to a static device scratch array
+ * of 2^21 floats (8 MiB) inside libmk.so, then are summed in a fixed order
+ * into C.  T * n_out must not exceed 2^21 (else MK_ERR_ARG); other argument
+ * rules and layouts as mk_debug_gemm.  The first call on a device (made
+ * with that device current) looks up the scratch address with
+ * cudaGetSymbolAddress; make that first call before any stream capture.
+ * Nothing needs to start at zero: every partial is written before it is
+ * read, and the private wait-error word starts at zero when the library
+ * loads.  Calls share the scratch, so calls that overlap (other streams or
+ * threads without ordering) race; serialise them. */
+int mk_debug_gemm_noalloc(const void *W, const void *X, float *C, int n_out,
+                          int T, int K, void *stream);
+
 /* Human-readable text of a status code. */
 const char *mk_strerror(int status);
 
