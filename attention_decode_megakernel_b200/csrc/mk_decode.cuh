@@ -23,10 +23,10 @@
 //    synchronises and delivers the vector; there is no grid barrier, no
 //    fence and no counter on the data path.  (The post's cooperative grid
 //    sync between layers is replaced by this data-driven wait.)
-//  * Seven consumer warps: bf16 GEMV rows (two per warp at a time) against an
-//    fp32 activation vector held in registers, the gated delta-rule row
+//  * Eleven consumer warps: bf16 GEMV rows (four per warp at a time) against
+//    the fp32 activation vector in shared memory, the gated delta-rule row
 //    update, split-K flash-decode attention with an online softmax and a
-//    last-CTA merge, SwiGLU, the tied LM head with a grid argmax.
+//    cooperative merge, SwiGLU, the tied LM head with a grid argmax.
 //  * Every wait is bounded by %globaltimer; on expiry the kernel records
 //    MK_ERR_TIMEOUT, runs the rest of its schedule without work, lets its
 //    in-flight copies land and returns.
@@ -36,7 +36,7 @@
 
 namespace mk {
 
-constexpr int NCW = 7;                  // consumer warps (8 warps per CTA: 255 registers each)
+constexpr int NCW = 11;                 // consumer warps (12 warps per CTA: 168 registers each)
 constexpr int NCT = NCW * 32;           // consumer threads
 constexpr int NTHR = NCT + 32;          // + producer warp
 constexpr int SLOT = 32768;             // ring slot bytes
@@ -112,7 +112,10 @@ __device__ __forceinline__ int att_splits(const DevModel& M, int pos) {
   return s < smax ? s : smax;
 }
 
-__device__ __forceinline__ PD describe(const DevModel& M, const StepArgs& a, int kind, int l,
+// Not inlined: the producer's two cursors and the consumer loop share one
+// copy, which keeps the kernel's instruction footprint (and instruction-cache
+// misses) down.
+__device__ __noinline__ PD describe(const DevModel& M, const StepArgs& a, int kind, int l,
                                        int gp, int cta, uint64_t pol_w, uint64_t pol_s) {
   PD d;
   d.p0 = d.p1 = nullptr;
@@ -975,7 +978,7 @@ struct ChunkCursor {
 };
 
 // Move to the first chunk at or after phase (l, p); skips empty phases.
-__device__ __forceinline__ void cursor_settle(ChunkCursor& c, const DevModel& M,
+__device__ __noinline__ void cursor_settle(ChunkCursor& c, const DevModel& M,
                                               const StepArgs& a, int cta, uint64_t pol_w,
                                               uint64_t pol_s) {
   while (true) {

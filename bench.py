@@ -220,6 +220,23 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(values, dist, device):
+    """Each timing as the maximum over all ranks (the slowest replica sets
+    the job's time); identity without a process group."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def replica_rate(world, units_per_rank, max_ms):
+    """Whole-job throughput of `world` independent replicas: every rank's
+    units over the slowest rank's time."""
+    return world * units_per_rank / (max_ms / 1000.0)
+
+
 def matrix_params(cfg):
     """Weights of every projection matrix of the layer stack (no embedding)."""
     import numpy as np
@@ -421,10 +438,7 @@ def main():
         dist.barrier()
     prefill_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
     decode_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
-    if dist:
-        t = torch.tensor([prefill_ms, decode_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        prefill_ms, decode_ms = float(t[0]), float(t[1])
+    prefill_ms, decode_ms = max_over_ranks([prefill_ms, decode_ms], dist, "cuda")
     out_tokens = toks.cpu().numpy().tolist()
 
     # end to end through the public API with host buffers: the first token
@@ -442,17 +456,13 @@ def main():
         host_toks.copy_(toks, non_blocking=True)
         stream.synchronize()
         e2e_times.append(time.perf_counter() - t0)
-    e2e_s = sum(e2e_times)
-    if dist:
-        t = torch.tensor([e2e_s], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t[0])
+    e2e_s = max_over_ranks([sum(e2e_times)], dist, "cuda")[0]
 
     hbm, _, peak_kind = peaks()
     per_launch_s = decode_ms / 1000.0 / (GEN * args.steps)
     bytes_avg = sum(decode_bytes(cfg, PROMPT + i) for i in range(GEN)) / GEN
     achieved = bytes_avg / per_launch_s / 1e9
-    value = world * GEN * args.steps / (decode_ms / 1000.0)
+    value = replica_rate(world, GEN * args.steps, decode_ms)
     prefill_tps = world * PROMPT * args.steps / (prefill_ms / 1000.0)
 
     cpu = None
