@@ -51,7 +51,7 @@ constexpr int CONV_ROWS_MAX = 256;      // in-projection rows of one CTA (conv s
 // words per consumer thread when NCT threads gather n tagged values
 constexpr int per_thread(int n) { return (n + NCT - 1) / NCT; }
 
-enum PhaseKind { PH_DN_IN, PH_DN_ST, PH_OUT, PH_Q, PH_K, PH_V, PH_ATT, PH_GU, PH_DOWN, PH_LM };
+enum PhaseKind { PH_DN_IN, PH_DN_ST, PH_OUT, PH_QKV, PH_ATT, PH_GU, PH_DOWN, PH_LM };
 
 struct StepArgs {
   DevModel m;         // the engine (by value: read through the constant bank)
@@ -144,19 +144,9 @@ __device__ __noinline__ PD describe(const DevModel& M, const StepArgs& a, int ki
       d.p0 = (const char*)(L.is_attn ? L.w_o : L.out_proj);
       d.row_bytes = (L.is_attn ? M.nq * M.hd : M.nh * M.dv) * 2;
       break;
-    case PH_Q:
-      balanced(M.nq * M.hd, idx, M.ncta, r0, r1);
-      d.p0 = (const char*)L.w_q;
-      d.row_bytes = M.H * 2;
-      break;
-    case PH_K:
-      balanced(M.nkv * M.hd, idx, M.ncta, r0, r1);
-      d.p0 = (const char*)L.w_k;
-      d.row_bytes = M.H * 2;
-      break;
-    case PH_V:
-      balanced(M.nkv * M.hd, idx, M.ncta, r0, r1);
-      d.p0 = (const char*)L.w_v;
+    case PH_QKV:  // q, k and v rows as one matrix (the engine's packed copy)
+      balanced((M.nq + 2 * M.nkv) * M.hd, idx, M.ncta, r0, r1);
+      d.p0 = (const char*)L.w_qkv;
       d.row_bytes = M.H * 2;
       break;
     case PH_GU:
@@ -202,9 +192,8 @@ __device__ __noinline__ PD describe(const DevModel& M, const StepArgs& a, int ki
 // Phase sequence of one layer.
 __device__ __forceinline__ int layer_phases(const DevLayer& L, int* kinds) {
   if (L.is_attn) {
-    kinds[0] = PH_Q; kinds[1] = PH_K; kinds[2] = PH_V; kinds[3] = PH_ATT;
-    kinds[4] = PH_OUT; kinds[5] = PH_GU; kinds[6] = PH_DOWN;
-    return 7;
+    kinds[0] = PH_QKV; kinds[1] = PH_ATT; kinds[2] = PH_OUT; kinds[3] = PH_GU; kinds[4] = PH_DOWN;
+    return 5;
   }
   kinds[0] = PH_DN_IN; kinds[1] = PH_DN_ST; kinds[2] = PH_OUT; kinds[3] = PH_GU; kinds[4] = PH_DOWN;
   return 5;
@@ -760,7 +749,7 @@ template <int HD, int GQ>
 __device__ __forceinline__ void attention_phase(const DevModel& M, const StepArgs& a,
                                                 const DevLayer& L, const PD& d, uint32_t& g,
                                                 unsigned char* ring, SmemTail* t, float* uni,
-                                                uint32_t tag_q, uint32_t tag_k, uint32_t tag_v,
+                                                uint32_t tag_qkv, uint32_t tag_dbg,
                                                 uint32_t tag_out, bool dry, int tid, int warp,
                                                 int lane) {
   constexpr int EPL = HD / 32;
@@ -779,9 +768,9 @@ __device__ __forceinline__ void attention_phase(const DevModel& M, const StepArg
     // raw q of the group's heads (staged in att_acc) and, for the split that
     // owns the new position, its raw k and v: one polling round
     const LLSeg sg[3] = {
-        {M.qkv_ll + gidx * G * HD, att_acc, G * HD, tag_q},
-        {M.qkv_ll + M.nq * HD + gidx * HD, att_kn, last ? HD : 0, tag_k},
-        {M.qkv_ll + (M.nq + M.nkv) * HD + gidx * HD, att_vn, last ? HD : 0, tag_v}};
+        {M.qkv_ll + gidx * G * HD, att_acc, G * HD, tag_qkv | tag_dbg},
+        {M.qkv_ll + M.nq * HD + gidx * HD, att_kn, last ? HD : 0, tag_qkv},
+        {M.qkv_ll + (M.nq + M.nkv) * HD + gidx * HD, att_vn, last ? HD : 0, tag_qkv}};
     ok = ll_gather_segs<per_thread(GQ * HD + 2 * HD), 3>(sg, t, M.err, a.wait_ns, tid);
   }
   const bool bad = named_sync_or(1, NCT, !ok);
@@ -1114,7 +1103,7 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
   int gp = 0;
   int kinds[8];
   // tags of the latest producer of each tagged buffer
-  uint32_t tag_x = 0, tag_inp = 0, tag_dno = 0, tag_q = 0, tag_k = 0, tag_v = 0, tag_att = 0,
+  uint32_t tag_x = 0, tag_inp = 0, tag_dno = 0, tag_qkv = 0, tag_att = 0,
            tag_h = 0;
   int xb = 0;  // residual buffer holding the latest x
 
@@ -1139,7 +1128,7 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
       bool gemv = false;
       switch (kind) {
         case PH_DN_IN:
-        case PH_Q:
+        case PH_QKV:
         case PH_GU:
         case PH_LM: {
           // input: RMSNorm of the residual stream (the embedding at layer 0)
@@ -1182,10 +1171,10 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
             j.conv_out = conv_g;
             j.ch = M.ch;
             tag_inp = tag_me;
-          } else if (kind == PH_Q) {
+          } else if (kind == PH_QKV) {
             j.epi = EPI_STORE;
-            j.dst = M.qkv_ll;
-            tag_q = tag_me;
+            j.dst = M.qkv_ll;  // [q | k | v], the rows' order
+            tag_qkv = tag_me;
           } else if (kind == PH_GU) {
             j.epi = EPI_SWIGLU;
             j.dst = M.mlph_ll;
@@ -1194,15 +1183,6 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
             j.epi = EPI_LOGITS;
             j.logits = a.logits;
           }
-          break;
-        }
-        case PH_K:
-        case PH_V: {
-          gemv = true;
-          j.epi = EPI_STORE;
-          j.dst = M.qkv_ll + (kind == PH_K ? M.nq * HD : (M.nq + M.nkv) * HD);
-          if (kind == PH_K) tag_k = tag_me;
-          else tag_v = tag_me;
           break;
         }
         case PH_OUT: {
@@ -1276,7 +1256,7 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
           tag_dno = tag_me;
           break;
         case PH_ATT:
-          attention_phase<HD, GQ>(M, a, L, d, g, ring, t, uni, tag_q | dbg, tag_k, tag_v, tag_me,
+          attention_phase<HD, GQ>(M, a, L, d, g, ring, t, uni, tag_qkv, dbg, tag_me,
                                   dry, tid, warp, lane);
           tag_att = tag_me;
           break;

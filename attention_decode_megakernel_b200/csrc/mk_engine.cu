@@ -24,6 +24,7 @@ struct Layout {
   size_t dn_state[mk::kStateBufs], conv_state[mk::kStateBufs];
   size_t kc, vc;
   size_t x, inp, dno, qkv, atto, mlph, part, hidden, logits, tickets, err, amax;
+  size_t wqkv;  // packed q|k|v weight rows of every attention layer
   // multi-token prompt path: T_MAX positions per chunk
   int tmax, pw, aw;
   size_t pf_tok, pf_x, pf_xn, pf_p, pf_c, pf_o, pf_a16, pf_qk, pf_bak, pf_att;
@@ -71,6 +72,7 @@ Layout make_layout(const mk_config& c) {
   const size_t kv = size_t(n_attn) * c.kv_heads * c.max_ctx * c.head_dim * 2;
   L.kc = take(kv);
   L.vc = take(kv);
+  L.wqkv = take(size_t(n_attn) * (c.q_heads + 2 * c.kv_heads) * c.head_dim * c.hidden * 2);
   L.x = take(2 * M * c.hidden * 8);
   L.inp = take(M * rin * 8);
   L.dno = take(M * c.dn_heads * c.dn_dv * 8);
@@ -557,6 +559,7 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
     D.w_k = static_cast<const uint16_t*>(L.w_k);
     D.w_v = static_cast<const uint16_t*>(L.w_v);
     D.w_o = static_cast<const uint16_t*>(L.w_o);
+    D.w_qkv = nullptr;
     D.mlp_norm = static_cast<const uint16_t*>(L.mlp_norm);
     D.w_gate = static_cast<const uint16_t*>(L.w_gate);
     D.w_up = static_cast<const uint16_t*>(L.w_up);
@@ -571,6 +574,27 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
   }
   m.kc = reinterpret_cast<uint16_t*>(ws + lay.kc);
   m.vc = reinterpret_cast<uint16_t*>(ws + lay.vc);
+  {
+    // the decode kernel reads each attention layer's q, k and v rows as one
+    // matrix: pack them once into the workspace
+    const size_t H2 = size_t(c.hidden) * 2;
+    const size_t qb = size_t(c.q_heads) * c.head_dim * H2, kb = size_t(c.kv_heads) * c.head_dim * H2;
+    for (int l = 0; l < c.n_layers; ++l) {
+      mk::DevLayer& D = m.layers[l];
+      if (!D.is_attn) continue;
+      char* dst = ws + lay.wqkv + size_t(D.sub) * (qb + 2 * kb);
+      cudaError_t r = cudaMemcpyAsync(dst, D.w_q, qb, cudaMemcpyDeviceToDevice, e->stream);
+      if (r == cudaSuccess)
+        r = cudaMemcpyAsync(dst + qb, D.w_k, kb, cudaMemcpyDeviceToDevice, e->stream);
+      if (r == cudaSuccess)
+        r = cudaMemcpyAsync(dst + qb + kb, D.w_v, kb, cudaMemcpyDeviceToDevice, e->stream);
+      if (r != cudaSuccess) {
+        delete e;
+        return cuda_status(r);
+      }
+      D.w_qkv = reinterpret_cast<const uint16_t*>(dst);
+    }
+  }
   using ull = unsigned long long;
   m.x_ll = reinterpret_cast<ull*>(ws + lay.x);
   m.inp_ll = reinterpret_cast<ull*>(ws + lay.inp);

@@ -17,6 +17,7 @@ struct DevLayer {
   const float *A_log, *dt_bias;
   const uint16_t *out_norm, *out_proj;
   const uint16_t *w_q, *w_k, *w_v, *w_o;
+  const uint16_t* w_qkv;  // engine copy of q|k|v rows, [(nq + 2 nkv) hd][H]
   const uint16_t *mlp_norm, *w_gate, *w_up, *w_down;
   int is_attn;
   int sub;  // index among layers of the same kind

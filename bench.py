@@ -27,6 +27,10 @@ sys.path.insert(0, ROOT)
 
 PROMPT = 520
 GEN = 128
+# DRAM bytes (read + written) of one decode launch at context 520, from an ncu
+# capture of the current decode kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum); None once the kernel changes.
+DECODE_TRAFFIC_BYTES = 1.3195e9
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -490,7 +494,7 @@ def main():
         "prefill_tok_s": prefill_tps,
         "decode_ms_per_token": per_launch_s * 1000.0,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None, "peak_kind": peak_kind,
+                     "frac": achieved / hbm, "traffic": DECODE_TRAFFIC_BYTES, "peak_kind": peak_kind,
                      "kernel": "decode_kernel (one launch per token)",
                      "bytes_per_launch": bytes_avg},
         "e2e": {"value": world * GEN * args.steps / e2e_s, "unit": "tok/s",

@@ -98,7 +98,8 @@ typedef struct {
 typedef struct mk_engine mk_engine;
 
 /* Bytes of device workspace mk_create needs for this config (recurrent
- * state, verify checkpoints, KV cache, activations, barrier words).
+ * state, verify checkpoints, KV cache, activations, exchange words, and a
+ * packed copy of each attention layer's q|k|v weight rows).
  * Returns 0 for an invalid config. */
 size_t mk_workspace_bytes(const mk_config *cfg);
 
@@ -108,7 +109,10 @@ size_t mk_workspace_bytes(const mk_config *cfg);
  * keeps pointers.  `cuda_stream` (a cudaStream_t, may be NULL for the
  * legacy stream) is the stream every later call runs on.  Checks that one
  * CTA of the decode kernel fits on every SM (cooperative co-residency) and
- * returns MK_ERR_LAUNCH otherwise.  Zeroes the state (as mk_reset). */
+ * returns MK_ERR_LAUNCH otherwise.  Copies each attention layer's w_q, w_k
+ * and w_v into one [q|k|v][hidden] block of the workspace (the decode
+ * kernel reads them as one matrix), so later changes to those three weights
+ * need a new engine.  Zeroes the state (as mk_reset). */
 int mk_create(const mk_config *cfg, const mk_weights *w, void *workspace,
               size_t ws_bytes, void *cuda_stream, mk_engine **out);
 
@@ -204,8 +208,8 @@ int64_t mk_launch_count(const mk_engine *e);
  * wait or a wait for another CTA's data that exceeds it records
  * MK_ERR_TIMEOUT and the kernel returns early.  `fail_phase` >= 0 makes the
  * next decode launch wait, in that phase (0-based index of the launch's
- * phase sequence: five phases per DeltaNet layer, seven per attention
- * layer), for data tagged with a value no phase ever writes, so the wait
+ * phase sequence: five phases per layer, then the LM head), for data
+ * tagged with a value no phase ever writes, so the wait
  * must run out (tests of the timeout path only). */
 int mk_debug_set_wait_limit(mk_engine *e, int64_t limit_ns, int fail_phase);
 

@@ -138,6 +138,28 @@ def test_08b_decode_after_state_load(mk, big):
     print(tr.finish())
 
 
+@pytest.mark.slow
+def test_08b_decode_at_32k_context(mk):
+    """Long-context shape: the attention layers' cache holds 32,768
+    positions (a seeded synthetic state of that shape) and the attention
+    split covers all of them; 2 teacher-forced steps against the oracle."""
+    cfg = synth.hybrid_08b_config(max_ctx=32768 + 8)
+    w = synth.make_weights(cfg)
+    st = synth.make_engine_state(cfg, ctx=32768)
+    eng = mk.Engine(cfg, w)
+    dev = {k: (torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v).cuda()
+               if isinstance(v, np.ndarray) else v) for k, v in st.items()}
+    eng.set_state(dev)
+    del dev
+    orc = oracle.OracleModel(cfg, w)
+    orc.set_state(st)
+    del st
+    tr = Tracker()
+    _teacher_forced(eng, orc, cfg, 4321, 2, tr)
+    _check_state(eng, orc)
+    print(tr.finish())
+
+
 def test_08b_prompt_then_decode(mk, big):
     cfg, w = big
     eng = mk.Engine(cfg, w)
@@ -268,13 +290,14 @@ def test_engine_errors(mk):
     assert e.value.code == mk.MK_ERR_ARG
 
 
-@pytest.mark.parametrize("phase", [1, 3, 9, 18, 19, 22])
+@pytest.mark.parametrize("phase", [1, 3, 9, 15, 16, 19, 20])
 def test_wait_limit_reports_timeout_and_recovers(mk, phase):
     """A phase whose inputs wait for a tag nobody writes must give up after the
     wait limit, report MK_ERR_TIMEOUT and leave the context usable; mk_reset
-    recovers the engine.  Tiny model phases: 1 DeltaNet state update, 3 first
-    MLP gate/up, 9 second layer's down projection, 18 attention (queries),
-    19 attention output projection, 22 LM head."""
+    recovers the engine.  Tiny model phases (five per layer): 1 DeltaNet
+    state update, 3 first MLP gate/up, 9 second layer's down projection,
+    15 attention q|k|v projection, 16 attention, 19 attention layer's down
+    projection, 20 LM head."""
     cfg = synth.tiny_config(max_ctx=64)
     w = synth.make_weights(cfg)
     eng = mk.Engine(cfg, w)
