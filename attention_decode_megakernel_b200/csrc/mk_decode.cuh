@@ -370,32 +370,46 @@ __device__ __forceinline__ void fma8x2(const uint4 w, const float* x, float& a, 
   b = fmaf(bf_hi(w.w), x[7], b);
 }
 
-// This lane's partial dot products of four rows (in shared memory) with the
+// This lane's partial dot products of R rows (in shared memory) with the
 // activation (shared memory): lane l takes 16-byte vectors l, l+32, ... of
-// each row and the matching 8 activation floats, read once for the four
-// rows.  One runtime loop serves every row length: the kernel runs each
-// phase's code once per token, so a compact instruction footprint beats
-// per-length unrolled copies.
-__device__ __forceinline__ void dot4(const unsigned char* r0, const unsigned char* r1,
-                                     const unsigned char* r2, const unsigned char* r3,
-                                     const float* xs, int nvec, int lane, float (&acc)[4]) {
-  const uint4* w0 = reinterpret_cast<const uint4*>(r0);
-  const uint4* w1 = reinterpret_cast<const uint4*>(r1);
-  const uint4* w2 = reinterpret_cast<const uint4*>(r2);
-  const uint4* w3 = reinterpret_cast<const uint4*>(r3);
-  float s[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+// each row and the matching 8 activation floats, read once for the R rows.
+// One runtime loop serves every row length: the kernel runs each phase's
+// code once per token, so a compact instruction footprint beats per-length
+// unrolled copies.
+template <int R>
+__device__ __forceinline__ void dot_rows(const unsigned char* const (&rows)[4], const float* xs,
+                                         int nvec, int lane, float (&acc)[R]) {
+  const uint4* w[R];
+#pragma unroll
+  for (int q = 0; q < R; ++q) w[q] = reinterpret_cast<const uint4*>(rows[q]);
+  float s[R][2];
+#pragma unroll
+  for (int q = 0; q < R; ++q) s[q][0] = s[q][1] = 0.f;
   for (int idx = lane; idx < nvec; idx += 32) {
     const float4 p = reinterpret_cast<const float4*>(xs)[idx * 2];
-    const float4 q = reinterpret_cast<const float4*>(xs)[idx * 2 + 1];
-    const float x[8] = {p.x, p.y, p.z, p.w, q.x, q.y, q.z, q.w};
-    const uint4 u0 = w0[idx], u1 = w1[idx], u2 = w2[idx], u3 = w3[idx];
-    fma8x2(u0, x, s[0][0], s[0][1]);
-    fma8x2(u1, x, s[1][0], s[1][1]);
-    fma8x2(u2, x, s[2][0], s[2][1]);
-    fma8x2(u3, x, s[3][0], s[3][1]);
+    const float4 h = reinterpret_cast<const float4*>(xs)[idx * 2 + 1];
+    const float x[8] = {p.x, p.y, p.z, p.w, h.x, h.y, h.z, h.w};
+    uint4 u[R];
+#pragma unroll
+    for (int q = 0; q < R; ++q) u[q] = w[q][idx];
+#pragma unroll
+    for (int q = 0; q < R; ++q) fma8x2(u[q], x, s[q][0], s[q][1]);
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q) acc[q] = s[q][0] + s[q][1];
+  for (int q = 0; q < R; ++q) acc[q] = s[q][0] + s[q][1];
+}
+
+// Warp reduction of two values at once: lanes 0-15 end with the sum of a,
+// lanes 16-31 with the sum of b (5 shuffles instead of 10).
+__device__ __forceinline__ float reduce2(float a, float b, int lane) {
+  const bool h16 = (lane & 16) != 0;
+  float x = h16 ? b : a;
+  x += __shfl_xor_sync(0xffffffffu, h16 ? a : b, 16);
+  x += __shfl_xor_sync(0xffffffffu, x, 8);
+  x += __shfl_xor_sync(0xffffffffu, x, 4);
+  x += __shfl_xor_sync(0xffffffffu, x, 2);
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  return x;
 }
 
 // ---- matrix phases ------------------------------------------------------------
@@ -457,11 +471,12 @@ __device__ __forceinline__ void gemv_epilogue(const GemvJob& j, int row, float y
 }
 
 // Walk the CTA's chunks of one matrix phase.  Each warp takes its rows of a
-// chunk four at a time (rows i, i+NCW, i+2NCW, i+3NCW; for EPI_SWIGLU the
-// gate and up rows of i and i+NCW), reduces the four dot products in one
-// transposed shuffle tree and parks each result in lane (count of results
-// so far); the epilogue then runs once per 32 results with every lane
-// finishing its own row, instead of one lane finishing rows one by one.
+// chunk up to four at a time (rows i, i+NCW, i+2NCW, i+3NCW; for EPI_SWIGLU
+// the gate and up rows of i and i+NCW), computes only the dot products of
+// rows that exist, reduces them in one transposed shuffle tree and parks
+// each result in lane (count of results so far); the epilogue then runs once
+// per 32 results with every lane finishing its own row, instead of one lane
+// finishing rows one by one.
 // The activation vector is in shared memory (xs).  Returns the chunk counter
 // after the phase.
 __device__ __forceinline__ uint32_t gemv_core(const GemvJob& j, uint32_t g, unsigned char* ring,
@@ -502,24 +517,43 @@ __device__ __forceinline__ uint32_t gemv_core(const GemvJob& j, uint32_t g, unsi
           p2 = base + size_t(nout > 2 ? i + 2 * NCW : i) * rb;
           p3 = base + size_t(nout > 3 ? i + 3 * NCW : i) * rb;
         }
-        float acc[4];
-        dot4(p0, p1, p2, p3, xs, nvec, lane, acc);
-        const float z = reduce4(acc[0], acc[1], acc[2], acc[3], lane);
+        // as many row dot products as this iteration has rows (a slot holds
+        // few rows per warp, so most iterations have one or two)
+        const unsigned char* const rows[4] = {p0, p1, p2, p3};
+        const int R = swiglu ? 2 * nout : (nout == 3 ? 4 : nout);
+        float z;
+        int sh;  // result q of the reduction sits in lanes q << sh ...
+        if (R == 1) {
+          float a1[1];
+          dot_rows<1>(rows, xs, nvec, lane, a1);
+          z = warp_sum(a1[0]);
+          sh = 5;
+        } else if (R == 2) {
+          float a2[2];
+          dot_rows<2>(rows, xs, nvec, lane, a2);
+          z = reduce2(a2[0], a2[1], lane);
+          sh = 4;
+        } else {
+          float a4[4];
+          dot_rows<4>(rows, xs, nvec, lane, a4);
+          z = reduce4(a4[0], a4[1], a4[2], a4[3], lane);
+          sh = 3;
+        }
         if (nb + nout > 32) {
           if (lane < nb) gemv_epilogue(j, krow, kv, kv2, best_v, best_i);
           nb = 0;
         }
         const int q = lane - nb;
-        if (swiglu) {
-          const float gv = __shfl_sync(0xffffffffu, z, (q & 1) << 4);
-          const float uv = __shfl_sync(0xffffffffu, z, ((q & 1) << 4) + 8);
+        if (swiglu) {  // results 2o (gate) and 2o+1 (up) of output o
+          const float gv = __shfl_sync(0xffffffffu, z, (2 * (q & 1)) << sh);
+          const float uv = __shfl_sync(0xffffffffu, z, (2 * (q & 1) + 1) << sh);
           if (q >= 0 && q < nout) {
             kv = gv;
             kv2 = uv;
             krow = r + i + q * NCW;
           }
         } else {
-          const float v = __shfl_sync(0xffffffffu, z, (q & 3) << 3);
+          const float v = __shfl_sync(0xffffffffu, z, (q & (R - 1)) << sh);
           if (q >= 0 && q < nout) {
             kv = v;
             krow = r + i + q * NCW;
