@@ -12,7 +12,7 @@
 //  * Each CTA owns a balanced slice of every phase (rows of each matrix,
 //    rows of the recurrent state, a split of the KV cache).  The slices are
 //    known at launch, so one producer warp walks the CTA's whole per-token
-//    byte stream and keeps a 6 x 32 KB shared-memory ring full with bulk TMA
+//    byte stream and keeps a 3 x 64 KB shared-memory ring full with bulk TMA
 //    copies (cp.async.bulk + mbarrier complete_tx).  It never waits for
 //    other CTAs: weights, the previous token's state rows and cached KV
 //    positions of later phases keep streaming while the consumers wait.
@@ -39,8 +39,8 @@ namespace mk {
 constexpr int NCW = 11;                 // consumer warps (12 warps per CTA: 168 registers each)
 constexpr int NCT = NCW * 32;           // consumer threads
 constexpr int NTHR = NCT + 32;          // + producer warp
-constexpr int SLOT = 32768;             // ring slot bytes
-constexpr int NSLOT = 6;                // ring slots
+constexpr int SLOT = 65536;             // ring slot bytes (more rows per slot: more rows per warp)
+constexpr int NSLOT = 3;                // ring slots
 constexpr int ATT_MIN_POS = 32;         // fewest positions per attention split
 constexpr int XRAW_MAX = 2048;          // largest hidden size (residual copy in shared memory)
 constexpr int UNION_FLOATS = 4096;      // activation vector | head cache | attention scratch
