@@ -900,8 +900,15 @@ int mk_debug_gemm(const void* W, const void* X, float* C, int n_out, int T, int 
   if (!make_map(&g.tw, W, n_out, K, K, mk::pf::BM) ||
       !make_map(&g.tx, X, 2 * T, K, K, mk::pf::BN))
     return MK_ERR_UNSUPPORTED;
-  static int* err_word = nullptr;
-  if (!err_word && cudaMalloc(&err_word, 4) != cudaSuccess) return MK_ERR_CUDA;
+  // a 4-byte wait-error word per device, allocated by the first call there
+  static int* err_words[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return MK_ERR_CUDA;
+  }
+  if (!err_words[dev] && cudaMalloc(&err_words[dev], 4) != cudaSuccess) return MK_ERR_CUDA;
+  int* err_word = err_words[dev];
   if (cudaFuncSetAttribute(mk::pf::gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            int(mk::pf::GEMM_SMEM)) != cudaSuccess)
     return MK_ERR_CUDA;

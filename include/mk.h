@@ -236,8 +236,9 @@ int mk_delta_step(float *S, const void *q, const void *k, const void *v,
  *   hi = bf16(x), lo = bf16(x - hi)); C device float32 [T][n_out]; all
  *   16-byte aligned, K a multiple of 64.
  * MK_ERR_ARG on bad sizes, MK_ERR_UNSUPPORTED if the TMA descriptors cannot
- * be encoded.  A device-side wait that runs out is recorded in a word
- * private to this call (not reported). */
+ * be encoded.  The first call on a device allocates a 4-byte device word
+ * (kept for the life of the process) where a device-side wait that runs
+ * out is recorded; it is not reported. */
 int mk_debug_gemm(const void *W, const void *X, float *C, int n_out, int T,
                   int K, void *stream);
 
