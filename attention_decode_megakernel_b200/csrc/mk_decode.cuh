@@ -986,7 +986,7 @@ __device__ __forceinline__ void attention_phase(const DevModel& M, const StepArg
 // Cursor over one CTA's chunk schedule for one launch: every phase of every
 // layer, then the LM head, each split into chunks of at most `rpc` rows.
 // ----------------------------------------------------------------------------
-constexpr size_t PF_AHEAD = size_t(128) << 10;  // L2 prefetch distance per CTA (bytes)
+constexpr size_t PF_AHEAD = size_t(64) << 10;  // L2 prefetch distance per CTA (bytes)
 
 struct ChunkCursor {
   int l, p, np, gp;
