@@ -30,7 +30,7 @@ GEN = 128
 # DRAM bytes (read + written) of one decode launch at context 520, from an ncu
 # capture of the current decode kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum); None once the kernel changes.
-DECODE_TRAFFIC_BYTES = 1.3193e9
+DECODE_TRAFFIC_BYTES = 1.3223e9
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
