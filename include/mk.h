@@ -50,11 +50,12 @@ typedef enum {
 } mk_status;
 
 /* Model shape.  Layer l is full attention when layer_is_attn[l] != 0 and a
- * Gated-DeltaNet layer otherwise.  Shapes the kernels implement:
- * hidden % 256 == 0 and <= 2048; dn_dk == dn_dv in {64, 128};
- * head_dim in {64, 128, 256}; conv_k == 4; q_heads % kv_heads == 0 and
- * q_heads / kv_heads <= 8; mlp % 8 == 0; the embedding is tied to the
- * LM head.  mk_create returns MK_ERR_UNSUPPORTED otherwise. */
+ * Gated-DeltaNet layer otherwise.  Shapes the decode kernel is built for:
+ * hidden % 256 == 0 and <= 2048; conv_k == 4; mlp % 8 == 0 and <= 4096; the embedding
+ * tied to the LM head; q_heads == 4 * kv_heads; and (dn_dk == dn_dv,
+ * head_dim) one of (64, 64), (128, 128), (128, 256).  mk_create returns
+ * MK_ERR_UNSUPPORTED otherwise (also when a CTA's share of a phase exceeds
+ * the kernel's shared-memory staging). */
 typedef struct {
   int32_t n_layers;
   uint8_t layer_is_attn[MK_MAX_LAYERS];
