@@ -183,6 +183,45 @@ def oracle_decode_rate(cfg, w, budget_s=12.0, max_steps=64):
     return n / dt, n, dt, cores
 
 
+def oracle_other_rates(cfg, w):
+    """The oracle on the other configurations, on small bounded samples (a
+    reported CPU baseline, not a target): prompt positions/s of the 0.8B
+    model (8 positions from an empty state; the oracle has no batched prompt
+    path, so this equals its decode rate at short context), verify calls/s
+    (5 positions from a cloned state at context 520, the oracle's
+    checkpoint = a clone) and gated delta steps/s for one sequence of
+    16 heads x 128 x 128 (64 steps)."""
+    import numpy as np
+    import oracle
+    from attention_decode_megakernel_b200 import synth
+    out = {}
+    m = oracle.OracleModel(cfg, w)
+    toks = synth.make_tokens(cfg.vocab, 8)
+    t0 = time.perf_counter()
+    for t in toks:
+        m.step(int(t), want_logits=False)
+    out["prefill_positions_s"] = len(toks) / (time.perf_counter() - t0)
+    m.set_state(synth.make_engine_state(cfg, ctx=PROMPT))
+    drafts = synth.make_tokens(cfg.vocab, 5, seed=synth.SEED_DRAFTS)
+    t0 = time.perf_counter()
+    c = m.clone()
+    for t in drafts:
+        c.step(int(t))
+    out["verify_calls_s"] = 1.0 / (time.perf_counter() - t0)
+    sw = synth.make_delta_sweep(1, 64, heads=16, dk=128, dv=128)
+    S = sw["S0"].astype(np.float64)
+    q = synth.bf16_bits_to_f32(sw["q"]).astype(np.float64)
+    k = synth.bf16_bits_to_f32(sw["k"]).astype(np.float64)
+    v = synth.bf16_bits_to_f32(sw["v"]).astype(np.float64)
+    t0 = time.perf_counter()
+    for h in range(16):
+        oracle.delta_sequence(S[0, h], q[:, 0, h], k[:, 0, h], v[:, 0, h],
+                              sw["alpha"][:, 0, h].astype(np.float64),
+                              sw["beta"][:, 0, h].astype(np.float64))
+    out["delta_steps_s_B1"] = 64 / (time.perf_counter() - t0)
+    return out
+
+
 def run_reference(args, rank):
     """Reference arm: the CPU oracle as it stands, on the host cores."""
     if rank != 0:
@@ -474,7 +513,8 @@ def main():
         rate, n, dt, cores = oracle_decode_rate(cfg, w)
         cpu = {"value": rate, "unit": "tok/s", "cores": cores, "kind": "oracle",
                "sample": "%d greedy decode steps of the 0.8B-shaped model at context 520 "
-                         "(seeded synthetic state) in %.1f s, fp64 oracle" % (n, dt)}
+                         "(seeded synthetic state) in %.1f s, fp64 oracle" % (n, dt),
+               "other_configs": oracle_other_rates(cfg, w)}
 
     extras = None
     if rank == 0 and world == 1 and not args.no_extras:
