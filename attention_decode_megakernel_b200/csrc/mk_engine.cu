@@ -27,12 +27,14 @@ struct Layout {
   size_t wqkv;  // packed q|k|v weight rows of every attention layer
   // multi-token prompt path: T_MAX positions per chunk
   int tmax, pw, aw;
-  size_t pf_tok, pf_x, pf_xn, pf_p, pf_c, pf_o, pf_a16, pf_qk, pf_bak, pf_att;
+  size_t pf_tok, pf_x, pf_xn, pf_p, pf_c, pf_o, pf_a16, pf_qk, pf_bak, pf_att, pf_part;
   size_t total;
 };
 
 constexpr int kPrefillChunk = 1024;  // most positions one prompt chunk processes
 constexpr int kPrefillMinBatch = 8;  // shorter prompts run as decode steps
+constexpr int kSplitMaxTiles = 100;      // prompt GEMMs with fewer output tiles split K
+constexpr int kSplitPartialTiles = 148 + kSplitMaxTiles;
 
 int count_attn(const mk_config& c) {
   int n = 0;
@@ -109,6 +111,9 @@ Layout make_layout(const mk_config& c) {
     // key-split attention partials of a short chunk: [t][q head][range][hd + 2]
     const size_t nsplit = (size_t(c.max_ctx) + mk::pf::ATT_SPLIT_LEN - 1) / mk::pf::ATT_SPLIT_LEN;
     L.pf_att = take(size_t(mk::kMaxVerify) * c.q_heads * nsplit * (c.head_dim + 2) * 4);
+    // split-K partial sums of a prompt GEMM with few output tiles (< 100):
+    // k_split x T x n_out <= (148 + tiles) x 128 x 128 floats
+    L.pf_part = take(size_t(kSplitPartialTiles) * mk::pf::BM * mk::pf::BN * 4);
   }
   L.total = off;
   return L;
@@ -260,9 +265,35 @@ int launch_decode(mk_engine* e, int pos, int st_buf, int token, int tok_src, flo
 int launch_gemm(mk_engine* e, const CUtensorMap& tw, const CUtensorMap& tx, float* c, int ldc,
                 int n_out, int T, int K, int accumulate) {
   const int tiles = ((n_out + mk::pf::BM - 1) / mk::pf::BM) * ((T + mk::pf::BN - 1) / mk::pf::BN);
-  int ks = T <= mk::pf::BN ? (e->ncta + tiles - 1) / tiles : 1;  // short chunks only
+  int ks = T <= mk::pf::BN || tiles < kSplitMaxTiles ? (e->ncta + tiles - 1) / tiles : 1;
   if (ks > K / mk::pf::BK) ks = K / mk::pf::BK;
   if (ks < 1) ks = 1;
+  if (ks > 1 && T > mk::pf::BN) {
+    // a prompt chunk: the ranges' sums go to partial buffers and are added
+    // in a fixed order by a second kernel (deterministic, no atomics)
+    mk::pf::GemmArgs g;
+    g.tw = tw;
+    g.tx = tx;
+    g.c = c;
+    g.ldc = ldc;
+    g.n_out = n_out;
+    g.T = T;
+    g.K = K;
+    g.accumulate = accumulate;
+    g.x_lo_row = e->lay.tmax;
+    g.k_split = ks;
+    g.err = e->hm.err;
+    g.wait_ns = e->wait_ns;
+    float* part = reinterpret_cast<float*>(e->ws + e->lay.pf_part);
+    const dim3 grid((n_out + mk::pf::BM - 1) / mk::pf::BM, (T + mk::pf::BN - 1) / mk::pf::BN, ks);
+    mk::pf::gemm_tc_partial<<<grid, mk::pf::GEMM_THREADS, mk::pf::GEMM_SMEM, e->stream>>>(g, part);
+    const size_t n = size_t(T) * n_out;
+    const int rb = int((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+    mk::pf::splitk_reduce_ld_kernel<<<rb, 256, 0, e->stream>>>(part, ks, T, n_out, c, ldc,
+                                                               accumulate);
+    e->launches += 2;
+    return cuda_status(cudaGetLastError());
+  }
   if (ks > 1 && !accumulate) {
     const cudaError_t r =
         cudaMemset2DAsync(c, size_t(ldc) * 4, 0, size_t(n_out) * 4, T, e->stream);
@@ -617,6 +648,9 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
   }
   // tensor maps of the prompt path (weights and the chunk's bf16 activations)
   e->pf_ok = cudaFuncSetAttribute(mk::pf::gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(mk::pf::GEMM_SMEM)) == cudaSuccess &&
+             cudaFuncSetAttribute(mk::pf::gemm_tc_partial,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   int(mk::pf::GEMM_SMEM)) == cudaSuccess;
   cudaGetLastError();
   {

@@ -280,6 +280,20 @@ __global__ void splitk_reduce_kernel(const float* partial, int k_split, size_t n
   }
 }
 
+// c[t][n] (+)= sum over z of partial[z][t][n] (z = 0, 1, ... in order), for
+// a split-K GEMM whose output has row stride ldc.
+__global__ void splitk_reduce_ld_kernel(const float* partial, int k_split, int T, int n_out,
+                                        float* c, int ldc, int accumulate) {
+  const size_t n = size_t(T) * n_out;
+  for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += size_t(gridDim.x) * blockDim.x) {
+    float acc = 0.f;
+    for (int z = 0; z < k_split; ++z) acc += partial[size_t(z) * n + i];
+    float* dst = c + (i / n_out) * size_t(ldc) + (i % n_out);
+    *dst = accumulate ? *dst + acc : acc;
+  }
+}
+
 // ---- elementwise / row kernels --------------------------------------------------
 constexpr int ROW_THREADS = 256;
 
