@@ -9,9 +9,10 @@
  * learned recurrence interleaved with full-attention layers; the kernel
  * bullet list: one dispatch for the whole forward pass, bf16 weights,
  * fp32 accumulation, fused QKV + RoPE + causal softmax + output
- * projection, cooperative grid sync between layers).  The recurrence is
- * the gated delta rule of "Gated Delta Networks" (Yang, Kautz &
- * Hatamizadeh, ICLR 2025).
+ * projection; the post synchronises the grid between layers, this engine
+ * lets each CTA wait for exactly the data it needs instead).  The
+ * recurrence is the gated delta rule of "Gated Delta Networks" (Yang,
+ * Kautz & Hatamizadeh, ICLR 2025).
  *
  * Conventions shared by all entry points
  *  - Every pointer documented as "device" must point to memory of the CUDA
@@ -19,11 +20,11 @@
  *    before the call returns.
  *  - Calls are asynchronous on the stream given to mk_create unless stated.
  *  - Nothing throws across the ABI.  Every call returns an mk_status code;
- *    MK_OK is 0.  A device-side failure (a grid barrier or pipeline wait
- *    that ran out of time) is recorded in a device error word and reported
- *    by mk_sync(), and by the next call that synchronises.  After any error
- *    the engine accepts only mk_reset() and mk_destroy(); mk_reset() clears
- *    the error, the recurrent state and the KV cache.
+ *    MK_OK is 0.  A device-side failure (a wait for another CTA's data or
+ *    a pipeline wait that ran out of time) is recorded in a device error
+ *    word and reported by mk_sync() until mk_reset() clears it; results of
+ *    calls made after such an error are undefined until then.  mk_reset()
+ *    clears the error, the recurrent state and the KV cache.
  *  - Tensors are row-major.  bf16 values are IEEE bfloat16 bit patterns.
  */
 #ifndef MK_H
@@ -131,28 +132,37 @@ int mk_reset(mk_engine *e);
  * "pp520" beside decode).  When n-1 >= 8 the first n-1 positions run as
  * chunks of up to 1024 positions: every projection one tensor-core GEMM
  * (bf16 weights; each fp32 activation as a bf16 hi + lo pair; fp32
- * accumulation), the
- * causal conv and gated delta rule scanned position by position, causal
- * attention over cache + chunk.  The last position is always one decode
- * step, so its logits and greedy argmax come from the decode kernel.
- * If logits_out (device, float32 [vocab]) is not NULL it receives the
- * logits of the last prompt position.  n == 0 is a no-op.
- * Errors: MK_ERR_CTX_OVERFLOW when pos+n > max_ctx. */
+ * accumulation), the causal conv and gated delta rule scanned position by
+ * position, causal attention over cache + chunk.  The last position is
+ * always one decode step, so its logits and greedy argmax come from the
+ * decode kernel.  If logits_out (device, float32 [vocab]) is not NULL it
+ * receives the logits of the last prompt position.  n == 0 is a no-op.
+ * The host array is copied before the call returns (pageable copies
+ * synchronise with the stream).  Errors: MK_ERR_ARG (token out of range),
+ * MK_ERR_CTX_OVERFLOW when pos+n > max_ctx, MK_ERR_STATE while a verify is
+ * pending, MK_ERR_LAUNCH / MK_ERR_CUDA on launch failures. */
 int mk_prefill(mk_engine *e, const int32_t *tokens_host, int n,
                float *logits_out);
 
-/* One decode step: one cooperative launch of the persistent kernel for
- * `token` at the current position.  logits_out (device, float32 [vocab])
- * may be NULL.  The greedy argmax of the step is kept on the device (see
- * mk_generate) and can be read with mk_last_argmax. */
+/* One decode step: the whole forward pass of `token` at the current
+ * position in one cooperative launch of the persistent kernel (launch post
+ * "OS Megakernel that match M5 Max Tok/w at 2x the Throughput on RTX 3090",
+ * kernel bullet list: one dispatch per token instead of ~100 launches).
+ * logits_out (device, float32 [vocab]) may be NULL.  The greedy argmax of
+ * the step is kept on the device (see mk_generate) and can be read with
+ * mk_last_argmax.  Does not synchronise the host.  Errors: MK_ERR_ARG
+ * (token out of range), MK_ERR_CTX_OVERFLOW at max_ctx, MK_ERR_STATE while
+ * a verify is pending, MK_ERR_LAUNCH / MK_ERR_CUDA on launch failures. */
 int mk_decode_step(mk_engine *e, int32_t token, float *logits_out);
 
-/* Greedy generation with no host round trip between tokens: n decode
- * launches, the first fed `first_token` (or, when first_token == -1, the
- * device-side argmax of the previous launch, e.g. the last prefill
- * position), each later one fed the device-side argmax of the launch before
- * it.  tokens_out (device, int32 [n]) receives
- * the n argmax tokens; logits_out (device, float32 [n][vocab]) may be NULL. */
+/* Greedy generation with no host round trip between tokens (the tg128
+ * decode of the launch post's results table): n decode launches, the first
+ * fed `first_token` (or, when first_token == -1, the device-side argmax of
+ * the previous launch, e.g. the last prefill position; MK_ERR_STATE if
+ * there was none), each later one fed the device-side argmax of the launch
+ * before it.  tokens_out (device, int32 [n]) receives the n argmax tokens;
+ * logits_out (device, float32 [n][vocab]) may be NULL.  Other errors as
+ * mk_decode_step. */
 int mk_generate(mk_engine *e, int32_t first_token, int n, int32_t *tokens_out,
                 float *logits_out);
 
