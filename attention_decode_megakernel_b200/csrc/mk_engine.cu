@@ -196,6 +196,7 @@ struct mk_engine {
   int cur_buf;
   uint32_t seq;  // launch sequence number for activation tags
   int amax_toggle;
+  bool amax_valid;  // the last launch was a decode step at the current position
   int pending_verify;
   int verify_bufs[mk::kMaxVerify];
   int64_t launches;
@@ -254,6 +255,7 @@ int launch_decode(mk_engine* e, int pos, int st_buf, int token, int tok_src, flo
     return MK_ERR_LAUNCH;
   }
   e->amax_toggle ^= 1;
+  e->amax_valid = true;
   e->launches += 1;
   return MK_OK;
 }
@@ -709,6 +711,7 @@ int mk_reset(mk_engine* e) {
   e->pos = 0;
   e->cur_buf = 0;
   e->amax_toggle = 0;
+  e->amax_valid = false;
   e->pending_verify = 0;
   return MK_OK;
 }
@@ -737,7 +740,7 @@ int mk_generate(mk_engine* e, int32_t first_token, int n, int32_t* tokens_out,
                 float* logits_out) {
   if (!e || n < 0 || !tokens_out) return MK_ERR_ARG;
   if (first_token < -1 || first_token >= e->cfg.vocab) return MK_ERR_ARG;
-  if (first_token == -1 && e->launches == 0) return MK_ERR_STATE;
+  if (first_token == -1 && !e->amax_valid) return MK_ERR_STATE;
   if (e->pending_verify) return MK_ERR_STATE;
   if (e->pos + n > e->cfg.max_ctx) return MK_ERR_CTX_OVERFLOW;
   for (int i = 0; i < n; ++i) {
@@ -790,6 +793,7 @@ int mk_verify(mk_engine* e, const int32_t* tokens_host, int n, float* logits_out
     const int rc = run_chunk(e, tokens_host, n, e->verify_bufs, logits_out);
     if (rc != MK_OK) return rc;
     e->pending_verify = n;
+    e->amax_valid = false;
     return MK_OK;
   }
   const Layout& L = e->lay;
@@ -812,6 +816,7 @@ int mk_verify(mk_engine* e, const int32_t* tokens_host, int n, float* logits_out
     ++k;
   }
   e->pending_verify = k;
+  e->amax_valid = false;  // the argmax is position n-1's; accept may keep fewer
   return MK_OK;
 }
 

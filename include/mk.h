@@ -158,9 +158,10 @@ int mk_decode_step(mk_engine *e, int32_t token, float *logits_out);
 /* Greedy generation with no host round trip between tokens (the tg128
  * decode of the launch post's results table): n decode launches, the first
  * fed `first_token` (or, when first_token == -1, the device-side argmax of
- * the previous launch, e.g. the last prefill position; MK_ERR_STATE if
- * there was none), each later one fed the device-side argmax of the launch
- * before it.  tokens_out (device, int32 [n]) receives the n argmax tokens;
+ * the last decode launch, which must be at the current position: the last
+ * prefill position or the last decode / generate step; MK_ERR_STATE after
+ * mk_create, mk_reset, mk_set_state or mk_verify), each later one fed the
+ * device-side argmax of the launch before it.  tokens_out (device, int32 [n]) receives the n argmax tokens;
  * logits_out (device, float32 [n][vocab]) may be NULL.  Other errors as
  * mk_decode_step. */
 int mk_generate(mk_engine *e, int32_t first_token, int n, int32_t *tokens_out,

@@ -290,6 +290,39 @@ def test_engine_errors(mk):
     assert e.value.code == mk.MK_ERR_ARG
 
 
+def test_engine_edge_cases(mk):
+    """Empty prompt, prompt past the cache, generate with no previous argmax,
+    verify while one is pending, accept counts out of range."""
+    cfg = synth.tiny_config(max_ctx=16)
+    w = synth.make_weights(cfg)
+    eng = mk.Engine(cfg, w)
+    toks = torch.zeros(4, dtype=torch.int32, device="cuda")
+    with pytest.raises(mk.MkError) as e:
+        eng.generate(-1, 4, toks)  # no launch yet: no device argmax to feed
+    assert e.value.code == mk.MK_ERR_STATE
+    eng.prefill([])
+    assert eng.position == 0
+    with pytest.raises(mk.MkError) as e:
+        eng.prefill(list(range(17)))
+    assert e.value.code == mk.MK_ERR_CTX_OVERFLOW
+    assert eng.position == 0
+    vl = torch.empty((3, cfg.vocab), dtype=torch.float32, device="cuda")
+    eng.verify([1, 2, 3], vl)
+    with pytest.raises(mk.MkError) as e:
+        eng.verify([1, 2, 3], vl)
+    assert e.value.code == mk.MK_ERR_STATE
+    with pytest.raises(mk.MkError) as e:
+        eng.decode_step(1)
+    assert e.value.code == mk.MK_ERR_STATE
+    for bad in (0, 4):
+        with pytest.raises(mk.MkError) as e:
+            eng.accept(bad)
+        assert e.value.code == mk.MK_ERR_ARG
+    eng.accept(3)
+    assert eng.position == 3
+    eng.sync()
+
+
 @pytest.mark.parametrize("phase", [1, 3, 9, 15, 16, 19, 20])
 def test_wait_limit_reports_timeout_and_recovers(mk, phase):
     """A phase whose inputs wait for a tag nobody writes must give up after the
