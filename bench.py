@@ -526,7 +526,7 @@ def main():
         "metric": "batch-1 decode tok/s (tg128)", "value": value, "unit": "tok/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": (prefill_ms + decode_ms) / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 weights, fp32 math",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "weights": "bf16",
         "data": "synthetic (seeded N(0,0.02) bf16 weights, uniform random prompt)",
         "config": {"workload": "hybrid-0.8B-24L-h1024 pp520+tg128", "prompt": PROMPT,
                    "gen": GEN, "batch": 1, "parallelism": "replicas" if world > 1 else "single",
