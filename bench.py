@@ -190,7 +190,8 @@ def oracle_other_rates(cfg, w):
     path, so this equals its decode rate at short context), verify calls/s
     (5 positions from a cloned state at context 520, the oracle's
     checkpoint = a clone) and gated delta steps/s for one sequence of
-    16 heads x 128 x 128 (64 steps)."""
+    16 heads x 128 x 128 (64 steps); the tiny model's decode tokens/s; the
+    0.8B decode on a single thread (2 steps)."""
     import numpy as np
     import oracle
     from attention_decode_megakernel_b200 import synth
@@ -219,6 +220,22 @@ def oracle_other_rates(cfg, w):
                               sw["alpha"][:, 0, h].astype(np.float64),
                               sw["beta"][:, 0, h].astype(np.float64))
     out["delta_steps_s_B1"] = 64 / (time.perf_counter() - t0)
+    # the tiny configuration's decode, and the 0.8B decode on one thread
+    tcfg = synth.tiny_config(max_ctx=64)
+    tm = oracle.OracleModel(tcfg, synth.make_weights(tcfg))
+    t0 = time.perf_counter()
+    for t in range(32):
+        tm.step(t)
+    out["tiny_decode_tok_s"] = 32 / (time.perf_counter() - t0)
+    oracle.set_threads(1)
+    try:
+        m.set_state(synth.make_engine_state(cfg, ctx=PROMPT))
+        t0 = time.perf_counter()
+        for t in range(2):
+            m.step(t + 1)
+        out["decode_tok_s_1_thread"] = 2 / (time.perf_counter() - t0)
+    finally:
+        oracle.set_threads(0)
     return out
 
 

@@ -69,6 +69,8 @@ def lib():
             getattr(L, f).restype = C.c_double
             getattr(L, f).argtypes = [C.c_double]
         L.orc_gemv.argtypes = [C.c_void_p, C.c_int, C.c_int, _D, _D]
+        L.orc_set_threads.argtypes = [C.c_int]
+        L.orc_set_threads.restype = None
         L.orc_rmsnorm.argtypes = [_D, C.c_void_p, C.c_int, C.c_double, _D]
         L.orc_l2norm.argtypes = [_D, C.c_int, C.c_double, _D]
         L.orc_causal_conv_step.argtypes = [C.c_int, C.c_int, C.c_void_p, _D, _D, _D]
@@ -111,6 +113,11 @@ def _vp(a):
 
 
 # ---- primitive wrappers (numpy in, numpy out) ----------------------------
+
+def set_threads(n: int):
+    """OpenMP threads for the oracle's GEMV rows (n <= 0: all cores)."""
+    lib().orc_set_threads(int(n))
+
 
 def sigmoid(x): return lib().orc_sigmoid(float(x))
 def softplus(x): return lib().orc_softplus(float(x))

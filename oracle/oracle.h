@@ -75,6 +75,9 @@ orc_model *orc_create(const orc_config *cfg, const orc_layer *layers,
                       const uint16_t *embed, const uint16_t *final_norm);
 orc_model *orc_clone(const orc_model *m);
 void orc_destroy(orc_model *m);
+/* Threads the independent GEMV rows may use (OpenMP; n <= 0: all cores).
+ * Only changes how fast the oracle runs, never what it computes. */
+void orc_set_threads(int n);
 void orc_reset(orc_model *m);
 int orc_pos(const orc_model *m);
 /* One token through the whole stack at position orc_pos(); logits [V] and
