@@ -23,6 +23,7 @@ MAX_LAYERS = 64
 
 MK_OK, MK_ERR_ARG, MK_ERR_CTX_OVERFLOW, MK_ERR_STATE = 0, 1, 2, 3
 MK_ERR_LAUNCH, MK_ERR_TIMEOUT, MK_ERR_CUDA, MK_ERR_UNSUPPORTED = 4, 5, 6, 7
+MK_ERR_RANGE = 8
 
 
 class MkError(RuntimeError):
@@ -87,6 +88,9 @@ def lib():
             "mk_debug_set_wait_limit": (C.c_int, [vp, i64, C.c_int]),
             "mk_delta_step": (C.c_int, [vp, vp, vp, vp, vp, vp, vp, C.c_int, C.c_int,
                                         C.c_int, C.c_int, vp]),
+            "mk_delta_chunked_ws_bytes": (sz, [C.c_int, C.c_int, C.c_int]),
+            "mk_delta_chunked": (C.c_int, [vp, vp, vp, vp, vp, vp, vp, C.c_int, C.c_int,
+                                           C.c_int, C.c_int, vp, sz, vp]),
             "mk_debug_gemm": (C.c_int, [vp, vp, vp, C.c_int, C.c_int, C.c_int, vp]),
             "mk_debug_gemm_noalloc": (C.c_int, [vp, vp, vp, C.c_int, C.c_int, C.c_int, vp]),
             "mk_strerror": (C.c_char_p, [C.c_int]),
@@ -270,6 +274,26 @@ def mk_delta_step(S, q, k, v, alpha, beta, o, stream=None):
     _check(lib().mk_delta_step(_ptr(S), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                                _ptr(o), int(B), int(heads), int(dk), int(dv), st),
            "mk_delta_step")
+
+
+def mk_delta_chunked(S, q, k, v, alpha, beta, o, workspace=None, stream=None):
+    """The gated delta rule over T positions in chunkwise form (in place on
+    S [heads][dv][dk]); q, k [heads][T][dk], v and o [heads][T][dv], alpha,
+    beta [heads][T], all float32 device tensors.  `workspace` (a device
+    tensor) may be given; otherwise one is allocated with torch."""
+    heads, dv, dk = S.shape
+    T = q.shape[1]
+    need = lib().mk_delta_chunked_ws_bytes(int(T), int(heads), int(dk))
+    if need == 0:
+        raise MkError(MK_ERR_ARG, "mk_delta_chunked_ws_bytes")
+    if workspace is None:
+        import torch
+        workspace = torch.empty(need, dtype=torch.uint8, device=S.device)
+    st = stream if stream is not None else 0
+    _check(lib().mk_delta_chunked(_ptr(S), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                  _ptr(o), int(T), int(heads), int(dk), int(dv), _ptr(workspace),
+                                  int(workspace.numel() * workspace.element_size()), st),
+           "mk_delta_chunked")
 
 
 def mk_debug_gemm(W, X, Cout, stream=None):

@@ -9,24 +9,32 @@
 // RoPE + causal softmax + output projection).
 //
 // B200 structure (differs from the post's 3090 design):
-//  * Each CTA owns a balanced slice of every phase (rows of each matrix,
-//    rows of the recurrent state, a split of the KV cache).  The slices are
-//    known at launch, so one producer warp walks the CTA's whole per-token
-//    byte stream and keeps a 3 x 64 KB shared-memory ring full with bulk TMA
-//    copies (cp.async.bulk + mbarrier complete_tx).  It never waits for
-//    other CTAs: weights, the previous token's state rows and cached KV
-//    positions of later phases keep streaming while the consumers wait.
-//  * Cross-CTA data travels as tagged words: every activation element another
-//    CTA needs is stored as one 8-byte word {fp32 value, 32-bit tag}, the tag
-//    naming the launch and the phase that produced it.  A consumer polls the
-//    words it needs until all tags match, so one L2 round trip both
-//    synchronises and delivers the vector; there is no grid barrier, no
-//    fence and no counter on the data path.  (The post's cooperative grid
-//    sync between layers is replaced by this data-driven wait.)
-//  * Eleven consumer warps: bf16 GEMV rows (four per warp at a time) against
-//    the fp32 activation vector in shared memory, the gated delta-rule row
-//    update, split-K flash-decode attention with an online softmax and a
-//    cooperative merge, SwiGLU, the tied LM head with a grid argmax.
+//  * The grid is split into ng groups of gs CTAs, one group per DeltaNet
+//    head (the 0.8B-shaped model: 16 groups of 9 CTAs; leftover SMs join
+//    the phases that are split over the whole grid).  A group computes its
+//    head's in-projection rows, exchanges them inside the group, and then
+//    every CTA of the group advances the head's whole recurrent state, so
+//    the readout and the gated norm need no further exchange.  Projections
+//    back to the residual stream (DeltaNet and attention output, MLP down)
+//    run split-K: group g owns K block g, its CTAs split the output rows,
+//    and the ng partial sums of each output meet in one 64-bit word per
+//    output (see "count-carrying sums" below).  The MLP's gate/up rows of
+//    K block g are computed inside group g and exchanged inside it.
+//  * Each CTA knows its share of every phase at launch, so one producer warp
+//    walks the CTA's whole per-token byte stream and keeps a 3 x 64 KB
+//    shared-memory ring full with bulk TMA copies (cp.async.bulk + mbarrier
+//    complete_tx).  It never waits for other CTAs.
+//  * Exchanges carry their own completion: a tagged word {fp32 value,
+//    32-bit tag naming launch and phase} for gathers, and for the split-K
+//    sums a word {8-bit count | 56-bit biased fixed-point sum} that every
+//    contributor adds to with one 64-bit atomic.  Integer addition makes the
+//    sum independent of arrival order (bit-reproducible), and a reader knows
+//    the sum is complete when the count equals the number of contributors.
+//    There is no grid barrier, no fence and no counter on the data path.
+//  * Eleven consumer warps: bf16 GEMV rows against fp32 activations in
+//    shared memory, the gated delta-rule row update, split-K flash-decode
+//    attention with an online softmax, SwiGLU, the tied LM head with a grid
+//    argmax.
 //  * Every wait is bounded by %globaltimer; on expiry the kernel records
 //    MK_ERR_TIMEOUT, runs the rest of its schedule without work, lets its
 //    in-flight copies land and returns.
@@ -36,22 +44,40 @@
 
 namespace mk {
 
-constexpr int NCW = 11;                 // consumer warps (12 warps per CTA: 168 registers each)
+constexpr int NCW = 11;                 // consumer warps (12 warps per CTA)
 constexpr int NCT = NCW * 32;           // consumer threads
 constexpr int NTHR = NCT + 32;          // + producer warp
-constexpr int SLOT = 65536;             // ring slot bytes (more rows per slot: more rows per warp)
+constexpr int SLOT = 65536;             // ring slot bytes
 constexpr int NSLOT = 3;                // ring slots
 constexpr int ATT_MIN_POS = 32;         // fewest positions per attention split
 constexpr int XRAW_MAX = 2048;          // largest hidden size (residual copy in shared memory)
 constexpr int UNION_FLOATS = 4096;      // activation vector | head cache | attention scratch
-constexpr int DN_HEADS_MAX = 4;         // heads one CTA's state rows may touch
-constexpr int DN_ROWS_MAX = 256;        // state rows of one CTA
 constexpr int CONV_ROWS_MAX = 256;      // in-projection rows of one CTA (conv staging)
+constexpr int MERGE_STAGE = 2048;       // partial values staged per attention-merge batch
+constexpr int MERGE_HEADS_MAX = 8;      // q heads one K block of the attention output spans
+constexpr int MERGE_ML_MAX = 1200;      // (m, l) words of all splits of those heads
+
+// count-carrying fixed-point sums: word = count << 56 | sum of (round(y * 2^32) + 2^46)
+constexpr int CFA_SHIFT = 56;
+constexpr unsigned long long CFA_MASK = (1ull << CFA_SHIFT) - 1;
+constexpr long long CFA_BIAS = 1ll << 46;
+constexpr double CFA_SCALE = 4294967296.0;  // 2^32
+constexpr float CFA_LIMIT = 8192.f;         // |contribution| < 2^13 keeps every sum in 56 bits
 
 // words per consumer thread when NCT threads gather n tagged values
 constexpr int per_thread(int n) { return (n + NCT - 1) / NCT; }
 
-enum PhaseKind { PH_DN_IN, PH_DN_ST, PH_OUT, PH_QKV, PH_ATT, PH_GU, PH_DOWN, PH_LM };
+enum PhaseKind {
+  PH_DN_IN,     // DeltaNet in-projection rows of the group's head (+ causal conv)
+  PH_DN_ST,     // the head's gated delta rule, readout and gated RMSNorm (whole head per CTA)
+  PH_DN_OUTP,   // DeltaNet output projection, K block = the group's head (split-K partial)
+  PH_QKV,       // attention q|k|v rows (whole grid)
+  PH_ATT,       // split-K flash-decode attention partials (whole grid)
+  PH_ATT_OUTP,  // merge of the partials of the group's K block + output projection partial
+  PH_GU,        // MLP gate/up rows of the group's K block of the hidden layer
+  PH_DOWNP,     // MLP down projection partial over the group's K block
+  PH_LM         // final norm + tied LM head rows (whole grid)
+};
 
 struct StepArgs {
   DevModel m;         // the engine (by value: read through the constant bank)
@@ -59,12 +85,12 @@ struct StepArgs {
   int token;          // input token when tok_src == 0
   int tok_src;        // 1: take the token from amax[amax_in]
   int amax_in, amax_out;
-  int st_buf;         // state buffer index
+  int st_in, st_out;  // state buffers read / written (distinct)
   float* logits;      // [V] (never NULL: scratch when the caller wants none)
   int32_t* tok_out;   // receives the argmax token (may be NULL)
   float* hidden;      // [n_layers][H] per-layer residual dump (may be NULL)
-  uint32_t seq;       // launch sequence number, 1 .. 2^23-1 (tag = seq << 8 | phase)
-  int fail_phase;     // debug: phase whose input tag can never match (-1 = none)
+  uint32_t seq;       // launch sequence number, 1 .. 2^23-1 (tag = seq << 9 | phase)
+  int fail_phase;     // debug: phase whose input can never complete (-1 = none)
   long long wait_ns;  // bound of every device-side wait
 };
 
@@ -80,15 +106,6 @@ struct __align__(16) SmemTail {
   unsigned long long best;
 };
 
-template <int DK, int HD, int GQ>
-struct Cfg {
-  static_assert(GQ * HD * 2 + 2 * HD + NCW * GQ * 2 <= UNION_FLOATS, "attention scratch");
-  static_assert(DN_HEADS_MAX * (2 * DK + 4) + 2 * DN_HEADS_MAX * DK + DN_ROWS_MAX +
-                    2 * DN_HEADS_MAX <= UNION_FLOATS,
-                "state-phase scratch");
-  static constexpr size_t SMEM =
-      size_t(NSLOT) * SLOT + sizeof(SmemTail) + (UNION_FLOATS + XRAW_MAX) * 4 + 128;
-};
 
 struct PD {                 // one CTA's share of one phase
   const char* p0;           // plane 0 base (row 0 of the phase's row space)
@@ -96,13 +113,26 @@ struct PD {                 // one CTA's share of one phase
   uint32_t row_bytes;       // bytes of one row of one plane
   int r0, n;                // first row and number of rows of this CTA
   int rpc;                  // rows per chunk
-  uint64_t pol;             // L2 policy of the copies
+  int keep;                 // 1: L2 evict-last copies (state, KV); 0: evict-first (weights)
   int unit_g, unit_s, S;    // attention split of this CTA (unit_g < 0: none)
 };
 
+constexpr int PHASES_PER_LAYER = 5;
+constexpr int MAX_PHASES = 128;  // schedule table entries (5 per layer + the LM head)
+
+template <int DK, int HD, int GQ>
+struct Cfg {
+  static_assert(GQ * HD * 2 + 2 * HD + NCW * GQ * 2 <= UNION_FLOATS, "attention scratch");
+  static_assert(4 * DK + 6 <= 2048 && 2048 + 2 * DK <= UNION_FLOATS - 256, "state-phase scratch");
+  static constexpr size_t SMEM = size_t(NSLOT) * SLOT + sizeof(SmemTail) +
+                                 (UNION_FLOATS + XRAW_MAX) * 4 + MAX_PHASES * sizeof(PD) + 128;
+};
+
+// Balanced split of n items into `parts`: [a, b) of part idx.  32-bit
+// arithmetic (n * parts < 2^32 for every split the kernel makes).
 __device__ __forceinline__ void balanced(int n, int idx, int parts, int& a, int& b) {
-  a = int((long long)n * idx / parts);
-  b = int((long long)n * (idx + 1) / parts);
+  a = int(unsigned(n) * unsigned(idx) / unsigned(parts));
+  b = int(unsigned(n) * unsigned(idx + 1) / unsigned(parts));
 }
 
 __device__ __forceinline__ int att_splits(const DevModel& M, int pos) {
@@ -112,56 +142,82 @@ __device__ __forceinline__ int att_splits(const DevModel& M, int pos) {
   return s < smax ? s : smax;
 }
 
-// Not inlined: the producer's two cursors and the consumer loop share one
-// copy, which keeps the kernel's instruction footprint (and instruction-cache
-// misses) down.
+// Group of a CTA (-1 for the CTAs beyond ng * gs) and its rotated index
+// inside the group for phase gp (rotation spreads the larger shares).
+__device__ __forceinline__ int group_of(const DevModel& M, int cta) {
+  return cta < M.ng * M.gs ? cta / M.gs : -1;
+}
+__device__ __forceinline__ int member_of(const DevModel& M, int cta, int gp) {
+  return (cta % M.gs + gp) % M.gs;
+}
+
+// One CTA's share of phase gp (layer l, kind).  Evaluated once per launch
+// for every phase, by as many threads as there are phases, into the schedule
+// table in shared memory that the producer and the consumers walk.
 __device__ __noinline__ PD describe(const DevModel& M, const StepArgs& a, int kind, int l,
-                                       int gp, int cta, uint64_t pol_w, uint64_t pol_s) {
+                                    int gp, int cta) {
   PD d;
   d.p0 = d.p1 = nullptr;
   d.row_bytes = 16;
-  d.pol = pol_w;
+  d.keep = 0;
   d.unit_g = -1;
   d.unit_s = 0;
   d.S = 0;
   const DevLayer& L = M.layers[l];
-  int idx = (cta + gp) % M.ncta;
+  const int grp = group_of(M, cta);
+  const int jj = member_of(M, cta, gp);
   int r0 = 0, r1 = 0;
   switch (kind) {
     case PH_DN_IN:
-      balanced(M.rin, idx, M.ncta, r0, r1);
-      d.p0 = (const char*)L.in_proj;
-      d.row_bytes = M.H * 2;
+      if (grp >= 0) {
+        balanced(M.rin_h, jj, M.gs, r0, r1);
+        d.p0 = (const char*)(L.w_in_pk + size_t(grp) * M.rin_h * M.H);
+        d.row_bytes = M.H * 2;
+      }
       break;
     case PH_DN_ST:
-      balanced(M.nh * M.dv, idx, M.ncta, r0, r1);
-      d.p0 = (const char*)(M.dn_state[a.st_buf] + size_t(L.sub) * M.nh * M.dv * M.dk);
-      d.row_bytes = M.dk * 4;
-      d.pol = pol_s;
+      if (grp >= 0) {
+        r0 = 0;
+        r1 = M.dv;
+        d.p0 = (const char*)(M.dn_state[a.st_in] + (size_t(L.sub) * M.nh + grp) * M.dv * M.dk);
+        d.row_bytes = M.dk * 4;
+        d.keep = 1;
+      }
       break;
-    case PH_OUT:
-      balanced(M.H, idx, M.ncta, r0, r1);
-      d.p0 = (const char*)(L.is_attn ? L.w_o : L.out_proj);
-      d.row_bytes = (L.is_attn ? M.nq * M.hd : M.nh * M.dv) * 2;
+    case PH_DN_OUTP:
+    case PH_ATT_OUTP: {
+      if (grp >= 0) {
+        const int kb = kind == PH_DN_OUTP ? M.dv : M.kb_att;
+        balanced(M.H, jj, M.gs, r0, r1);
+        d.p0 = (const char*)(L.w_out_blk + size_t(grp) * M.H * kb);
+        d.row_bytes = kb * 2;
+      }
       break;
+    }
     case PH_QKV:  // q, k and v rows as one matrix (the engine's packed copy)
-      balanced((M.nq + 2 * M.nkv) * M.hd, idx, M.ncta, r0, r1);
+      balanced((M.nq + 2 * M.nkv) * M.hd, (cta + gp) % M.ncta, M.ncta, r0, r1);
       d.p0 = (const char*)L.w_qkv;
       d.row_bytes = M.H * 2;
       break;
     case PH_GU:
-      balanced(M.I, idx, M.ncta, r0, r1);
-      d.p0 = (const char*)L.w_gate;
-      d.p1 = (const char*)L.w_up;
-      d.row_bytes = M.H * 2;
+      if (grp >= 0) {
+        balanced(M.kb_mlp, jj, M.gs, r0, r1);
+        r0 += grp * M.kb_mlp;
+        r1 += grp * M.kb_mlp;
+        d.p0 = (const char*)L.w_gate;
+        d.p1 = (const char*)L.w_up;
+        d.row_bytes = M.H * 2;
+      }
       break;
-    case PH_DOWN:
-      balanced(M.H, idx, M.ncta, r0, r1);
-      d.p0 = (const char*)L.w_down;
-      d.row_bytes = M.I * 2;
+    case PH_DOWNP:
+      if (grp >= 0) {
+        balanced(M.H, jj, M.gs, r0, r1);
+        d.p0 = (const char*)(L.w_down_blk + size_t(grp) * M.H * M.kb_mlp);
+        d.row_bytes = M.kb_mlp * 2;
+      }
       break;
     case PH_LM:
-      balanced(M.V, idx, M.ncta, r0, r1);
+      balanced(M.V, (cta + gp) % M.ncta, M.ncta, r0, r1);
       d.p0 = (const char*)M.embed;
       d.row_bytes = M.H * 2;
       break;
@@ -169,7 +225,7 @@ __device__ __noinline__ PD describe(const DevModel& M, const StepArgs& a, int ki
       int S = att_splits(M, a.pos);
       d.S = S;
       d.row_bytes = M.hd * 2;
-      d.pol = pol_s;
+      d.keep = 1;
       if (cta < M.nkv * S) {
         int g = cta / S, s = cta % S;
         d.unit_g = g;
@@ -189,13 +245,27 @@ __device__ __noinline__ PD describe(const DevModel& M, const StepArgs& a, int ki
   return d;
 }
 
+// Kind and layer of phase gp (PHASES_PER_LAYER per layer, then the LM head).
+__device__ __forceinline__ int phase_kind(const DevModel& M, int gp, int& l) {
+  l = gp / PHASES_PER_LAYER;
+  if (l >= M.n_layers) {
+    l = 0;
+    return PH_LM;
+  }
+  static constexpr int dn[PHASES_PER_LAYER] = {PH_DN_IN, PH_DN_ST, PH_DN_OUTP, PH_GU, PH_DOWNP};
+  static constexpr int at[PHASES_PER_LAYER] = {PH_QKV, PH_ATT, PH_ATT_OUTP, PH_GU, PH_DOWNP};
+  return M.layers[l].is_attn ? at[gp % PHASES_PER_LAYER] : dn[gp % PHASES_PER_LAYER];
+}
+
 // Phase sequence of one layer.
 __device__ __forceinline__ int layer_phases(const DevLayer& L, int* kinds) {
   if (L.is_attn) {
-    kinds[0] = PH_QKV; kinds[1] = PH_ATT; kinds[2] = PH_OUT; kinds[3] = PH_GU; kinds[4] = PH_DOWN;
+    kinds[0] = PH_QKV; kinds[1] = PH_ATT; kinds[2] = PH_ATT_OUTP; kinds[3] = PH_GU;
+    kinds[4] = PH_DOWNP;
     return 5;
   }
-  kinds[0] = PH_DN_IN; kinds[1] = PH_DN_ST; kinds[2] = PH_OUT; kinds[3] = PH_GU; kinds[4] = PH_DOWN;
+  kinds[0] = PH_DN_IN; kinds[1] = PH_DN_ST; kinds[2] = PH_DN_OUTP; kinds[3] = PH_GU;
+  kinds[4] = PH_DOWNP;
   return 5;
 }
 
@@ -232,7 +302,7 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, Sme
 }
 
 __device__ __forceinline__ uint32_t make_tag(uint32_t seq, int phase) {
-  return (seq << 8) | uint32_t(phase & 0xFF);
+  return (seq << 9) | uint32_t(phase & 0x1FF);
 }
 __device__ __forceinline__ void ll_put(unsigned long long* p, float v, uint32_t tag) {
   unsigned long long w = (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(v);
@@ -254,14 +324,16 @@ __device__ __forceinline__ bool ll_gather(float* dst, const unsigned long long* 
                                           long long wait_ns, int tid) {
   if (aborted(t)) return false;
   unsigned long long w[MAXK];
+#pragma unroll
+  for (int j = 0; j < MAXK; ++j) w[j] = static_cast<unsigned long long>(~tag) << 32;
   uint64_t start = 0;
   for (int it = 0;; ++it) {
 #pragma unroll
     for (int j = 0; j < MAXK; ++j) {
       const int i = tid + j * NCT;
-      unsigned long long v = static_cast<unsigned long long>(tag) << 32;
-      if (i < n) v = ll_get(src + i);
-      w[j] = v;
+      // words already seen complete are not polled again
+      if (i >= n) w[j] = static_cast<unsigned long long>(tag) << 32;
+      else if (uint32_t(w[j] >> 32) != tag) w[j] = ll_get(src + i);
     }
     bool stale = false;
 #pragma unroll
@@ -353,8 +425,111 @@ __device__ __forceinline__ bool ll_gather_segs(const LLSeg (&sg)[NSEG], SmemTail
   return true;
 }
 
+// All NCT consumer threads poll n tagged words (word i at addr(i)) until
+// every tag equals `tag`, then store the values to dst[i] (shared memory).
+// Each thread keeps its words in registers, so all its loads are in flight
+// at once, and re-reads only words still stale.  Uniform result.
+template <int MAXK, class AddrFn>
+__device__ __forceinline__ bool poll_words(float* dst, int n, AddrFn addr, uint32_t tag,
+                                           SmemTail* t, int* err, long long wait_ns, int tid) {
+  unsigned long long w[MAXK];
+#pragma unroll
+  for (int j = 0; j < MAXK; ++j) w[j] = static_cast<unsigned long long>(~tag) << 32;
+  uint64_t start = 0;
+  for (int it = 0;; ++it) {
+#pragma unroll
+    for (int j = 0; j < MAXK; ++j) {
+      const int i = tid + j * NCT;
+      if (i < n && uint32_t(w[j] >> 32) != tag) w[j] = ll_get(addr(i));
+    }
+    bool stale = false;
+#pragma unroll
+    for (int j = 0; j < MAXK; ++j) {
+      const int i = tid + j * NCT;
+      if (i < n) stale |= uint32_t(w[j] >> 32) != tag;
+    }
+    if (!named_sync_or(1, NCT, stale)) break;
+    if (it == 0) start = global_ns();
+    else if ((it & 7) == 0 && named_sync_or(1, NCT, give_up(t, err, start, wait_ns)))
+      return false;
+  }
+#pragma unroll
+  for (int j = 0; j < MAXK; ++j) {
+    const int i = tid + j * NCT;
+    if (i < n) dst[i] = __uint_as_float(uint32_t(w[j]));
+  }
+  return true;
+}
+
 // ----------------------------------------------------------------------------
-// GEMV helpers (a warp takes four rows at a time).  Lane l owns 16-byte
+// count-carrying fixed-point sums (the split-K reductions into the residual)
+// ----------------------------------------------------------------------------
+// Add one contribution y to the word at p.  A contribution outside the
+// fixed-point range (or not finite) records MK_ERR_RANGE and adds 0, so the
+// count still completes and no reader waits in vain.
+__device__ __forceinline__ void cfa_add(unsigned long long* p, float y, int* err) {
+  if (!(fabsf(y) < CFA_LIMIT)) {
+    record_error(err, MK_ERR_RANGE);
+    y = 0.f;
+  }
+  // y * 2^32 is exact in fp32 (|y| < 2^13), so its float-to-integer
+  // rounding is the rounding of y to the 2^-32 grid
+  const long long q = __float2ll_rn(y * 4294967296.0f);
+  const unsigned long long w =
+      (1ull << CFA_SHIFT) + static_cast<unsigned long long>(q + CFA_BIAS);
+  asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+
+// Consumer threads wait until each of the n words at src counts `want`
+// contributions, add the decoded sums to the residual xr[0..n) (shared
+// memory), and write xg = xr * gain (the RMSNorm numerator; gv are this
+// thread's gains) to xg, returning this thread's sum of xr^2.  Returns false
+// in *ok on timeout / abort (per thread; callers agree through
+// named_sync_or).
+template <int MAXK>
+__device__ __forceinline__ float cfa_read_add(float* xr, float* xg, const float* gv,
+                                              const unsigned long long* src, int n, int want,
+                                              SmemTail* t, int* err, long long wait_ns, int tid,
+                                              bool& ok) {
+  ok = false;
+  if (aborted(t)) return 0.f;
+  unsigned long long w[MAXK];
+#pragma unroll
+  for (int j = 0; j < MAXK; ++j) w[j] = 0;
+  uint64_t start = 0;
+  for (int it = 0;; ++it) {
+#pragma unroll
+    for (int j = 0; j < MAXK; ++j) {
+      const int i = tid + j * NCT;
+      if (i >= n) w[j] = static_cast<unsigned long long>(want) << CFA_SHIFT;
+      else if (int(w[j] >> CFA_SHIFT) != want) w[j] = ll_get(src + i);
+    }
+    bool stale = false;
+#pragma unroll
+    for (int j = 0; j < MAXK; ++j) stale |= int(w[j] >> CFA_SHIFT) != want;
+    if (!stale) break;
+    if (it == 0) start = global_ns();
+    else if ((it & 7) == 0 && give_up(t, err, start, wait_ns)) return 0.f;
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < MAXK; ++j) {
+    const int i = tid + j * NCT;
+    if (i < n) {
+      const long long q = static_cast<long long>(w[j] & CFA_MASK) - CFA_BIAS * want;
+      // the sum is a multiple of 2^-32: one rounding to fp32, exact scaling
+      const float v = xr[i] + __ll2float_rn(q) * (1.0f / 4294967296.0f);
+      xr[i] = v;
+      xg[i] = v * gv[j];
+      ss = fmaf(v, v, ss);
+    }
+  }
+  ok = true;
+  return ss;
+}
+
+// ----------------------------------------------------------------------------
+// GEMV helpers (a warp takes up to four rows at a time).  Lane l owns 16-byte
 // weight vectors v*32 + l of a row (8 bf16 each) and the matching 8
 // activation floats.
 // ----------------------------------------------------------------------------
@@ -416,49 +591,60 @@ __device__ __forceinline__ float reduce2(float a, float b, int lane) {
 // One routine serves every matrix phase, so the hot loop exists once in the
 // instruction stream (a phase switch then finds it cached); the epilogue is a
 // small runtime switch.
-enum EpiKind { EPI_STORE, EPI_RESID, EPI_INPROJ, EPI_SWIGLU, EPI_LOGITS };
+enum EpiKind { EPI_STORE, EPI_CFA, EPI_INPROJ, EPI_SWIGLU, EPI_LOGITS };
 
 struct GemvJob {
   PD d;
   int epi;                   // EpiKind
-  unsigned long long* dst;   // tagged destination, indexed by row
-  const float* xraw;         // EPI_RESID: residual before the update (shared memory)
-  float* hidden;             // EPI_RESID: optional per-layer dump
-  const float4* conv_s;      // EPI_INPROJ: conv history rows staged in shared memory
-  const uint2* conv_taps;    // EPI_INPROJ: conv taps rows staged in shared memory
-  float4* conv_out;          // EPI_INPROJ: the layer's conv history in global memory
-  int ch;                    // EPI_INPROJ: conv channels (rows below ch get the conv)
+  unsigned long long* dst;   // destination words, indexed by row - dst_off
+  int dst_off;
+  int* err;                  // EPI_CFA: range errors
+  const float4* conv_s;      // EPI_INPROJ: conv history of the CTA's rows (shared memory)
+  const uint2* conv_taps;    // EPI_INPROJ: conv taps of the CTA's rows (shared memory)
+  float4* conv_out;          // EPI_INPROJ: the layer's conv history in the output state buffer
+  int dk, nconv;             // EPI_INPROJ: head rows q|k|v below nconv get the conv
+  int chan_q, chan_k, chan_v;  // EPI_INPROJ: conv channels of the head's first q, k, v rows
+  int row_b;                 // EPI_INPROJ: packed rows row_b (b) and row_b + 1 (a) become the gates
+  float a_log, dt_bias;      // EPI_INPROJ: the head's decay parameters
   float* logits;             // EPI_LOGITS
+  float scale;               // multiplies every dot product (the RMSNorm factor)
   uint32_t tag;
 };
+
+// Conv channel of packed in-projection row p of one head (p < 2 dk + dv).
+__device__ __forceinline__ int conv_channel(const GemvJob& j, int p) {
+  return p < j.dk ? j.chan_q + p : p < 2 * j.dk ? j.chan_k + (p - j.dk) : j.chan_v + (p - 2 * j.dk);
+}
 
 __device__ __forceinline__ void gemv_epilogue(const GemvJob& j, int row, float y, float y2,
                                               float& best_v, int& best_i) {
   switch (j.epi) {
     case EPI_STORE:
-      ll_put(j.dst + row, y, j.tag);
+      ll_put(j.dst + (row - j.dst_off), y, j.tag);
       break;
-    case EPI_RESID: {
-      const float v = j.xraw[row] + y;
-      ll_put(j.dst + row, v, j.tag);
-      if (j.hidden) j.hidden[row] = v;
+    case EPI_CFA:
+      cfa_add(j.dst + (row - j.dst_off), y, j.err);
       break;
-    }
     case EPI_INPROJ:
-      if (row < j.ch) {
+      if (row < j.nconv) {
         // taps (u_{t-3}, u_{t-2}, u_{t-1}, u_t); shift the history by one
         const float4 s = j.conv_s[row - j.d.r0];
         const uint2 wc = j.conv_taps[row - j.d.r0];
         const float c =
             bf_lo(wc.x) * s.x + bf_hi(wc.x) * s.y + bf_lo(wc.y) * s.z + bf_hi(wc.y) * y;
-        j.conv_out[row] = make_float4(s.y, s.z, y, 0.f);
-        ll_put(j.dst + row, siluf_(c), j.tag);
+        j.conv_out[conv_channel(j, row)] = make_float4(s.y, s.z, y, 0.f);
+        ll_put(j.dst + (row - j.dst_off), siluf_(c), j.tag);
+      } else if (row == j.row_b) {
+        ll_put(j.dst + (row - j.dst_off), sigmoidf_(y), j.tag);  // beta
+      } else if (row == j.row_b + 1) {
+        // alpha = exp(-exp(A_log) * softplus(a + dt_bias))
+        ll_put(j.dst + (row - j.dst_off), expf(-expf(j.a_log) * softplusf_(y + j.dt_bias)), j.tag);
       } else {
-        ll_put(j.dst + row, y, j.tag);
+        ll_put(j.dst + (row - j.dst_off), y, j.tag);  // z
       }
       break;
     case EPI_SWIGLU:
-      ll_put(j.dst + row, siluf_(y) * y2, j.tag);
+      ll_put(j.dst + (row - j.dst_off), siluf_(y) * y2, j.tag);
       break;
     case EPI_LOGITS:
       j.logits[row] = y;
@@ -517,8 +703,7 @@ __device__ __forceinline__ uint32_t gemv_core(const GemvJob& j, uint32_t g, unsi
           p2 = base + size_t(nout > 2 ? i + 2 * NCW : i) * rb;
           p3 = base + size_t(nout > 3 ? i + 3 * NCW : i) * rb;
         }
-        // as many row dot products as this iteration has rows (a slot holds
-        // few rows per warp, so most iterations have one or two)
+        // as many row dot products as this iteration has rows
         const unsigned char* const rows[4] = {p0, p1, p2, p3};
         const int R = swiglu ? 2 * nout : (nout == 3 ? 4 : nout);
         float z;
@@ -540,7 +725,7 @@ __device__ __forceinline__ uint32_t gemv_core(const GemvJob& j, uint32_t g, unsi
           sh = 3;
         }
         if (nb + nout > 32) {
-          if (lane < nb) gemv_epilogue(j, krow, kv, kv2, best_v, best_i);
+          if (lane < nb) gemv_epilogue(j, krow, kv * j.scale, kv2 * j.scale, best_v, best_i);
           nb = 0;
         }
         const int q = lane - nb;
@@ -565,15 +750,71 @@ __device__ __forceinline__ uint32_t gemv_core(const GemvJob& j, uint32_t g, unsi
     __syncwarp();
     if (lane == 0) mbar_arrive(&t->empty[slot]);
   }
-  if (lane < nb) gemv_epilogue(j, krow, kv, kv2, best_v, best_i);
+  if (lane < nb) gemv_epilogue(j, krow, kv * j.scale, kv2 * j.scale, best_v, best_i);
   if (j.epi == EPI_LOGITS && best_i != 0x7FFFFFFF)
     atomicMax(&t->best, pack_argmax(best_v, best_i));
   return g;
 }
 
+// Matrix phases with short rows (the split-K partials, at most 64 16-byte
+// vectors per row): LPR lanes share a row, LPR the smallest power of two
+// that leaves each lane at most four vectors, so a warp takes 32 / LPR rows
+// at a time; the lane's activation slices stay in registers for the phase
+// and a row's sum needs log2(LPR) shuffles.
+__device__ __forceinline__ uint32_t gemv_short(const GemvJob& j, uint32_t g, unsigned char* ring,
+                                               SmemTail* t, int* err, long long wait_ns,
+                                               const float* xs) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const PD& d = j.d;
+  const int nvec = int(d.row_bytes / 16);
+  const int LPR = nvec <= 8 ? 2 : nvec <= 16 ? 4 : nvec <= 32 ? 8 : 16;
+  const int sl = lane & (LPR - 1), rpp = 32 / LPR, sub = lane / LPR;
+  float xr[4][8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int v = sl + LPR * k;
+    float4 p = make_float4(0.f, 0.f, 0.f, 0.f), h = p;
+    if (v < nvec) {
+      p = reinterpret_cast<const float4*>(xs)[v * 2];
+      h = reinterpret_cast<const float4*>(xs)[v * 2 + 1];
+    }
+    xr[k][0] = p.x; xr[k][1] = p.y; xr[k][2] = p.z; xr[k][3] = p.w;
+    xr[k][4] = h.x; xr[k][5] = h.y; xr[k][6] = h.z; xr[k][7] = h.w;
+  }
+  float bv = 0.f;
+  int bi = 0;
+#pragma unroll 1
+  for (int r = d.r0; r < d.r0 + d.n; r += d.rpc, ++g) {
+    const int slot = int(g % NSLOT);
+    if (bounded_wait(&t->full[slot], (g / NSLOT) & 1, t, err, wait_ns)) {
+      const int nr = min(d.rpc, d.r0 + d.n - r);
+      const unsigned char* base = ring + size_t(slot) * SLOT;
+#pragma unroll 1
+      for (int i0 = warp * rpp; i0 < nr; i0 += NCW * rpp) {
+        const int i = i0 + sub;
+        float a = 0.f, b = 0.f;
+        if (i < nr) {
+          const uint4* w = reinterpret_cast<const uint4*>(base + size_t(i) * d.row_bytes);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int v = sl + LPR * k;
+            if (v < nvec) fma8x2(w[v], xr[k], a, b);
+          }
+        }
+        float z = a + b;
+        for (int o = LPR / 2; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        if (i < nr && sl == 0) gemv_epilogue(j, r + i, z * j.scale, 0.f, bv, bi);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&t->empty[slot]);
+  }
+  return g;
+}
+
 // ----------------------------------------------------------------------------
-// RMSNorm of the vector already in `xin` (all NCT consumer threads):
-// xin = xin * rsqrt(mean(xin^2) + eps) * gain, keeping the raw copy in xraw.
+// RMSNorm: the GEMVs that read a normalised residual take x * gain as their
+// activation and scale every dot product by rsqrt(mean(x^2) + eps).
 // ----------------------------------------------------------------------------
 // Gains of RMSNorm as this thread uses them (element tid + k*NCT), loaded
 // before the input is awaited so their latency overlaps the wait.
@@ -584,33 +825,6 @@ __device__ __forceinline__ void load_gains(float (&gv)[GK], const uint16_t* gain
     const int i = tid + k * NCT;
     gv[k] = (gain && i < H) ? bf2f(gain[i]) : 1.f;
   }
-}
-
-__device__ __forceinline__ void rmsnorm_inplace(float* xin, float* xraw, const float (&gv)[GK],
-                                                int H, float eps, SmemTail* t, int tid) {
-  float ss = 0.f;
-#pragma unroll
-  for (int k = 0; k < GK; ++k) {
-    const int i = tid + k * NCT;
-    if (i < H) {
-      const float v = xin[i];
-      if (xraw) xraw[i] = v;
-      ss = fmaf(v, v, ss);
-    }
-  }
-  ss = warp_sum(ss);
-  if ((tid & 31) == 0) t->red[tid >> 5] = ss;
-  named_sync(1, NCT);
-  float tot = 0.f;
-#pragma unroll
-  for (int w = 0; w < NCW; ++w) tot += t->red[w];
-  const float inv = 1.0f / sqrtf(tot / float(H) + eps);
-#pragma unroll
-  for (int k = 0; k < GK; ++k) {
-    const int i = tid + k * NCT;
-    if (i < H) xin[i] = xin[i] * inv * gv[k];
-  }
-  named_sync(1, NCT);
 }
 
 // Chunk loop for the non-GEMV phases (state rows, KV positions): the body
@@ -639,101 +853,152 @@ __device__ __forceinline__ void rmsnorm_inplace(float* xin, float* xraw, const f
   } while (0)
 
 // ----------------------------------------------------------------------------
-// gated delta rule on this CTA's rows of the state (one layer, one token)
+// One DeltaNet head's gated delta rule, readout and gated RMSNorm (every CTA
+// of the head's group computes the whole head; each writes back its share
+// of the new state rows).  Head cache layout in uni (floats), as gathered:
+//   [0, DK) q   [DK, 2DK) k   [2DK, 2DK+dv) v   [2DK+dv, 2DK+2dv) z   then
+//   beta, alpha (computed by the in-projection epilogue)
+//   ov = uni + 2048: readout o (dv)   gv = uni + 2048 + DK: gated output (dv)
 // ----------------------------------------------------------------------------
 template <int DK>
 __device__ __forceinline__ void dn_state_phase(const DevModel& M, const StepArgs& a,
                                                const DevLayer& L, const PD& d, uint32_t& g,
                                                unsigned char* ring, SmemTail* t, float* uni,
-                                               uint32_t tag_in, uint32_t tag_out, bool dry,
-                                               int tid, int warp, int lane) {
+                                               uint32_t tag_in, bool dry, int grp, int tid,
+                                               int warp, int lane) {
   constexpr int EPL = DK / 32;
-  constexpr int stride = 2 * DK + 4;  // head cache: [q(dk) | k(dk) | beta, alpha, k.q, -]
-  const int h_first = d.n > 0 ? d.r0 / M.dv : 0;
-  const int n_heads = d.n > 0 ? (d.r0 + d.n - 1) / M.dv - h_first + 1 : 0;
-  // staging: raw q, k of the touched heads, v of this CTA's rows, b and a
-  float* sq_raw = uni + DN_HEADS_MAX * stride;   // [n_heads][DK]
-  float* sk_raw = sq_raw + DN_HEADS_MAX * DK;    // [n_heads][DK]
-  float* vrow = sk_raw + DN_HEADS_MAX * DK;      // [d.n]
-  float* sba = vrow + DN_ROWS_MAX;               // [2][n_heads]
+  float* hc = uni;
+  float* ov = uni + 2048;
+  float* gvec = uni + 2048 + DK;
   bool ok = true;
-  if (!dry && d.n > 0) {
-    const LLSeg sg[5] = {
-        {M.inp_ll + h_first * DK, sq_raw, n_heads * DK, tag_in},
-        {M.inp_ll + M.nh * DK + h_first * DK, sk_raw, n_heads * DK, tag_in},
-        {M.inp_ll + 2 * M.nh * DK + d.r0, vrow, d.n, tag_in},
-        {M.inp_ll + M.ch + M.nh * M.dv + h_first, sba, n_heads, tag_in},
-        {M.inp_ll + M.ch + M.nh * M.dv + M.nh + h_first, sba + DN_HEADS_MAX, n_heads, tag_in}};
-    ok = ll_gather_segs<per_thread(2 * DN_HEADS_MAX * DK + DN_ROWS_MAX + 2 * DN_HEADS_MAX), 5>(
-        sg, t, M.err, a.wait_ns, tid);
-  }
+  // the gated norm's gain (element tid), loaded before the wait
+  const float wgain = (grp >= 0 && tid < M.dv) ? bf2f(L.out_norm[tid]) : 0.f;
+  if (!dry && grp >= 0)
+    ok = ll_gather<per_thread(4 * DK + 2)>(hc, M.grp_inp + size_t(grp) * M.rin_h, M.rin_h,
+                                           tag_in, t, M.err, a.wait_ns, tid);
   const bool bad = named_sync_or(1, NCT, !ok);
-  if (!dry && !bad) {
-    for (int hh = warp; hh < n_heads; hh += NCW) {
-      const int h = h_first + hh;
-      float qv[EPL], kv[EPL];
-      float sq = 0.f, sk = 0.f;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        qv[e] = sq_raw[hh * DK + lane * EPL + e];
-        kv[e] = sk_raw[hh * DK + lane * EPL + e];
-        sq = fmaf(qv[e], qv[e], sq);
-        sk = fmaf(kv[e], kv[e], sk);
-      }
-      sq = warp_sum(sq);
-      sk = warp_sum(sk);
-      // q, k L2-normalised (eps 1e-6 inside the root); q also scaled by dk^-1/2
-      const float iq = 1.0f / sqrtf(sq + 1e-6f) / sqrtf(float(DK));
-      const float ik = 1.0f / sqrtf(sk + 1e-6f);
-      float kq = 0.f;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        qv[e] *= iq;
-        kv[e] *= ik;
-        kq = fmaf(kv[e], qv[e], kq);
-        uni[hh * stride + lane * EPL + e] = qv[e];
-        uni[hh * stride + DK + lane * EPL + e] = kv[e];
-      }
-      kq = warp_sum(kq);
-      if (lane == 0) {
-        const float b = sba[hh], aa = sba[DN_HEADS_MAX + hh];
-        uni[hh * stride + 2 * DK + 0] = sigmoidf_(b);  // beta
-        uni[hh * stride + 2 * DK + 1] =
-            expf(-expf(L.A_log[h]) * softplusf_(aa + L.dt_bias[h]));  // alpha
-        uni[hh * stride + 2 * DK + 2] = kq;
-      }
-    }
-  }
-  named_sync(1, NCT);
-  float* st = M.dn_state[a.st_buf] + size_t(L.sub) * M.nh * M.dv * DK;
-  MK_CHUNK_LOOP(d, {
-    const int h = row / M.dv;
-    const float* hc = uni + (h - h_first) * stride;
-    const float* sr = reinterpret_cast<const float*>(p0) + lane * EPL;
-    float sv[EPL], kv[EPL];
-    float s_k = 0.f, s_q = 0.f;
+  const bool work = !dry && !bad && grp >= 0;
+  // every warp normalises q and k itself (no serial step, no barrier):
+  // q, k L2-normalised (eps 1e-6 inside the root), q also scaled by dk^-1/2
+  float iq = 0.f, ik = 0.f, kq = 0.f;
+  if (work) {
+    float sq = 0.f, sk = 0.f, qk = 0.f;
 #pragma unroll
     for (int e = 0; e < EPL; ++e) {
-      sv[e] = sr[e];
-      kv[e] = hc[DK + lane * EPL + e];
-      s_k = fmaf(sv[e], kv[e], s_k);
-      s_q = fmaf(sv[e], hc[lane * EPL + e], s_q);
+      const float qv = hc[lane * EPL + e], kv = hc[DK + lane * EPL + e];
+      sq = fmaf(qv, qv, sq);
+      sk = fmaf(kv, kv, sk);
+      qk = fmaf(qv, kv, qk);
     }
-    s_k = warp_sum(s_k);
-    s_q = warp_sum(s_q);
-    const float beta = hc[2 * DK], alpha = hc[2 * DK + 1], kq = hc[2 * DK + 2];
-    const float u = beta * (vrow[row - d.r0] - alpha * s_k);  // S' = alpha S + u k^T
-    float* dst = st + size_t(row) * DK + lane * EPL;
-    if constexpr (EPL == 4) {
-      *reinterpret_cast<float4*>(dst) =
-          make_float4(fmaf(alpha, sv[0], u * kv[0]), fmaf(alpha, sv[1], u * kv[1]),
-                      fmaf(alpha, sv[2], u * kv[2]), fmaf(alpha, sv[3], u * kv[3]));
-    } else {
+    sq = warp_sum(sq);
+    sk = warp_sum(sk);
+    qk = warp_sum(qk);
+    iq = 1.0f / sqrtf(sq + 1e-6f) / sqrtf(float(DK));
+    ik = 1.0f / sqrtf(sk + 1e-6f);
+    kq = qk * iq * ik;
+    // w * SiLU(z) of the gated norm, completed after the rows (dv <= NCT)
+    if (tid < M.dv) gvec[tid] = wgain * siluf_(hc[2 * DK + M.dv + tid]);
+  }
+  // this CTA's share of the rows written back (the same split for every
+  // launch of the group, unrotated)
+  int w0 = 0, w1 = 0;
+  if (grp >= 0) balanced(M.dv, int(blockIdx.x) % M.gs, M.gs, w0, w1);
+  float* st = M.dn_state[a.st_out] + (size_t(L.sub) * M.nh + (grp < 0 ? 0 : grp)) * M.dv * DK;
+  const float beta = hc[4 * DK], alpha = hc[4 * DK + 1];  // gates from the in-projection
+  // The head's dv rows are one ring chunk.  Eight lanes share a row (a warp
+  // takes four rows at a time); sub-lane sl owns the float4 columns
+  // sl, sl + 8, ... so a row's eight lanes read consecutive 16-byte words
+  // (no bank conflicts), and k and q for those columns stay in registers.
+  constexpr int LPR = 8, V4 = DK / (4 * LPR);
+  const int sl = lane & (LPR - 1), ro = lane / LPR;
+  float4 kk[V4], qq[V4];
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) dst[e] = fmaf(alpha, sv[e], u * kv[e]);
+  for (int k = 0; k < V4; ++k) {
+    const float4 kr = reinterpret_cast<const float4*>(hc + DK)[sl + LPR * k];
+    const float4 qr = reinterpret_cast<const float4*>(hc)[sl + LPR * k];
+    kk[k] = make_float4(kr.x * ik, kr.y * ik, kr.z * ik, kr.w * ik);
+    qq[k] = make_float4(qr.x * iq, qr.y * iq, qr.z * iq, qr.w * iq);
+  }
+  float oss = 0.f;  // this lane's rows' o^2 (lanes with sl == 0)
+  if (d.n > 0) {
+    const int slot = int(g % NSLOT);
+    const bool okw = bounded_wait(&t->full[slot], (g / NSLOT) & 1, t, M.err, a.wait_ns);
+    if (okw && work) {
+      const float* base = reinterpret_cast<const float*>(ring + size_t(slot) * SLOT);
+      for (int r0 = warp * 4; r0 < d.n; r0 += NCW * 4) {
+        const int row = r0 + ro;
+        const bool has = row < d.n;
+        float4 sv[V4];
+        float s_k = 0.f, s_q = 0.f;
+#pragma unroll
+        for (int k = 0; k < V4; ++k) {
+          sv[k] = has ? reinterpret_cast<const float4*>(base + size_t(row) * DK)[sl + LPR * k]
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+          s_k = fmaf(sv[k].x, kk[k].x, s_k);
+          s_k = fmaf(sv[k].y, kk[k].y, s_k);
+          s_k = fmaf(sv[k].z, kk[k].z, s_k);
+          s_k = fmaf(sv[k].w, kk[k].w, s_k);
+          s_q = fmaf(sv[k].x, qq[k].x, s_q);
+          s_q = fmaf(sv[k].y, qq[k].y, s_q);
+          s_q = fmaf(sv[k].z, qq[k].z, s_q);
+          s_q = fmaf(sv[k].w, qq[k].w, s_q);
+        }
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1) {
+          s_k += __shfl_xor_sync(0xffffffffu, s_k, o);
+          s_q += __shfl_xor_sync(0xffffffffu, s_q, o);
+        }
+        if (has) {
+          const float u = beta * (hc[2 * DK + row] - alpha * s_k);  // S' = alpha S + u k^T
+          if (row >= w0 && row < w1) {
+            float4* dst = reinterpret_cast<float4*>(st + size_t(row) * DK);
+#pragma unroll
+            for (int k = 0; k < V4; ++k)
+              dst[sl + LPR * k] = make_float4(fmaf(alpha, sv[k].x, u * kk[k].x),
+                                              fmaf(alpha, sv[k].y, u * kk[k].y),
+                                              fmaf(alpha, sv[k].z, u * kk[k].z),
+                                              fmaf(alpha, sv[k].w, u * kk[k].w));
+          }
+          if (sl == 0) {
+            const float o = fmaf(alpha, s_q, u * kq);  // o_i = S'_i . q
+            ov[row] = o;
+            oss = fmaf(o, o, oss);
+          }
+        }
+      }
     }
-    if (lane == 0) ll_put(M.dno_ll + row, fmaf(alpha, s_q, u * kq), tag_out);  // o_i = S'_i.q
-  });
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&t->empty[slot]);
+    ++g;
+  }
+  oss = warp_sum(oss);
+  if (lane == 0) t->red[warp] = oss;
+  const bool skip = named_sync_or(1, NCT, !work || aborted(t));
+  if (skip) return;
+  // gated RMSNorm of the head's readout: g = o * rsqrt(mean(o^2) + eps) * w * SiLU(z)
+  float ss = 0.f;
+#pragma unroll
+  for (int w = 0; w < NCW; ++w) ss += t->red[w];
+  const float inv = 1.0f / sqrtf(ss / float(M.dv) + M.eps);
+  if (tid < M.dv) gvec[tid] *= ov[tid] * inv;
+  named_sync(1, NCT);
+}
+
+// EPL consecutive bf16 values (16, 8 or 4 bytes, aligned) as floats.
+template <int EPL>
+__device__ __forceinline__ void load_bf16_vec(const uint16_t* p, float (&f)[EPL]) {
+  if constexpr (EPL == 8) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    f[0] = bf_lo(u.x); f[1] = bf_hi(u.x); f[2] = bf_lo(u.y); f[3] = bf_hi(u.y);
+    f[4] = bf_lo(u.z); f[5] = bf_hi(u.z); f[6] = bf_lo(u.w); f[7] = bf_hi(u.w);
+  } else if constexpr (EPL == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    f[0] = bf_lo(u.x); f[1] = bf_hi(u.x); f[2] = bf_lo(u.y); f[3] = bf_hi(u.y);
+  } else {
+    static_assert(EPL == 2, "head_dim 64, 128 or 256");
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+    f[0] = bf_lo(u); f[1] = bf_hi(u);
+  }
 }
 
 // One key/value row into a warp's online-softmax state for G query heads
@@ -777,7 +1042,10 @@ __device__ __forceinline__ void att_consume(float (&am)[G], float (&al)[G], floa
 }
 
 // ----------------------------------------------------------------------------
-// split-K flash-decode attention for one KV group and position range
+// split-K flash-decode attention for one KV group and position range: the
+// CTA's partial (per q head of the group: accumulator, running max m and
+// denominator l) is published as tagged words; the merge happens in the
+// output-projection phase (att_merge_block).
 // ----------------------------------------------------------------------------
 template <int HD, int GQ>
 __device__ __forceinline__ void attention_phase(const DevModel& M, const StepArgs& a,
@@ -820,7 +1088,6 @@ __device__ __forceinline__ void attention_phase(const DevModel& M, const StepArg
   }
   named_sync(1, NCT);
   if (work) {
-    for (int i = tid; i < G * HD; i += NCT) att_acc[i] = 0.f;
     if (last) {
       // RoPE the new key, store K/V at `pos` in bf16, keep the rounded values
       const size_t cofs = ((size_t(L.sub) * M.nkv + gidx) * M.max_ctx + a.pos) * HD;
@@ -854,132 +1121,172 @@ __device__ __forceinline__ void attention_phase(const DevModel& M, const StepArg
     }
   }
   const float scale = 1.0f / sqrtf(float(HD));
-  MK_CHUNK_LOOP(d, {
-    const uint16_t* k16 = reinterpret_cast<const uint16_t*>(p0) + lane * EPL;
-    const uint16_t* v16 = reinterpret_cast<const uint16_t*>(p1) + lane * EPL;
-    float kf[EPL], vf[EPL];
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      kf[e] = bf2f(k16[e]);
-      vf[e] = bf2f(v16[e]);
+  // The chunk loop keeps the last ring slot: once its cached positions are
+  // consumed it is the scratch where the warps' partials are combined.
+  int keep_slot = -1;
+  {
+    int local_ = 0;
+    for (int r_ = d.r0; r_ < d.r0 + d.n; r_ += d.rpc, ++g, local_ += d.rpc) {
+      const int slot_ = int(g % NSLOT);
+      const bool ok_ = bounded_wait(&t->full[slot_], (g / NSLOT) & 1, t, M.err, a.wait_ns);
+      if (ok_) {
+        const int nr_ = min(d.rpc, d.r0 + d.n - r_);
+        const unsigned char* base_ = ring + size_t(slot_) * SLOT;
+        for (int i_ = (warp - (local_ % NCW) + NCW) % NCW; i_ < nr_; i_ += NCW) {
+          float kf[EPL], vf[EPL];
+          load_bf16_vec<EPL>(reinterpret_cast<const uint16_t*>(base_ + size_t(i_) * d.row_bytes) +
+                                 lane * EPL,
+                             kf);
+          load_bf16_vec<EPL>(
+              reinterpret_cast<const uint16_t*>(base_ + size_t(d.rpc + i_) * d.row_bytes) +
+                  lane * EPL,
+              vf);
+          att_consume<G, EPL>(am, al, acc, qr, kf, vf, scale);
+        }
+      }
+      __syncwarp();
+      if (r_ + d.rpc < d.r0 + d.n) {
+        if (lane == 0) mbar_arrive(&t->empty[slot_]);
+      } else {
+        keep_slot = slot_;
+      }
     }
-    att_consume<G, EPL>(am, al, acc, qr, kf, vf, scale);
-  });
-  const bool dry_post = named_sync_or(1, NCT, aborted(t) || !work);
-  if (dry_post) return;
-  // the new position (not in the cache at launch) goes to the next warp in turn
-  if (last && warp == (d.n % NCW)) {
-    float kf[EPL], vf[EPL];
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      kf[e] = att_kn[lane * EPL + e];
-      vf[e] = att_vn[lane * EPL + e];
-    }
-    att_consume<G, EPL>(am, al, acc, qr, kf, vf, scale);
   }
-  // combine the warps' (m, l, acc) into one partial for this split
-  if (lane == 0) {
+  const bool go = !named_sync_or(1, NCT, aborted(t) || !work);
+  if (go) {
+    // the new position (not in the cache at launch) goes to the next warp in turn
+    if (last && warp == (d.n % NCW)) {
+      float kf[EPL], vf[EPL];
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        kf[e] = att_kn[lane * EPL + e];
+        vf[e] = att_vn[lane * EPL + e];
+      }
+      att_consume<G, EPL>(am, al, acc, qr, kf, vf, scale);
+    }
+    // combine the warps' (m, l, acc) into one partial for this split
+    if (lane == 0) {
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        att_ml[(warp * G + j) * 2 + 0] = am[j];
+        att_ml[(warp * G + j) * 2 + 1] = al[j];
+      }
+    }
+    named_sync(1, NCT);
+    float fw[G];
 #pragma unroll
     for (int j = 0; j < G; ++j) {
-      att_ml[(warp * G + j) * 2 + 0] = am[j];
-      att_ml[(warp * G + j) * 2 + 1] = al[j];
+      float mx = -INFINITY;
+      for (int w = 0; w < NCW; ++w) mx = fmaxf(mx, att_ml[(w * G + j) * 2]);
+      fw[j] = al[j] > 0.f ? expf(am[j] - mx) : 0.f;
     }
-  }
-  named_sync(1, NCT);
-  // fixed warp order (deterministic): warp w adds its rescaled accumulator
-  float fw[G];
-#pragma unroll
-  for (int j = 0; j < G; ++j) {
-    float mx = -INFINITY;
-    for (int w = 0; w < NCW; ++w) mx = fmaxf(mx, att_ml[(w * G + j) * 2]);
-    fw[j] = al[j] > 0.f ? expf(am[j] - mx) : 0.f;
-  }
-  for (int w = 0; w < NCW; ++w) {
-    if (warp == w) {
+    // publish this split's partial as tagged words: per head [acc(HD) | m | l]
+    unsigned long long* pbase =
+        M.part_ll + (size_t(gidx) * kMaxCtas + d.unit_s) * G * (HD + 2);
+    if (keep_slot >= 0) {
+      // every warp's rescaled accumulator to the kept slot ([warp][head][HD],
+      // element lane*EPL + e at e*32 + lane: conflict-free), then one sum per
+      // element in warp order (deterministic)
+      float* scr = reinterpret_cast<float*>(ring + size_t(keep_slot) * SLOT);
 #pragma unroll
       for (int j = 0; j < G; ++j)
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) att_acc[j * HD + lane * EPL + e] += fw[j] * acc[j][e];
+        for (int e = 0; e < EPL; ++e) scr[(warp * G + j) * HD + e * 32 + lane] = fw[j] * acc[j][e];
+      named_sync(1, NCT);
+      for (int off = tid; off < G * HD; off += NCT) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < NCW; ++w) sum += scr[w * G * HD + off];
+        const int j = off / HD, rem = off % HD;
+        ll_put(pbase + j * (HD + 2) + (rem % 32) * EPL + rem / 32, sum, tag_out);
+      }
+    } else if (warp == 0) {
+      // no cached positions: warp 0 alone holds the new position
+#pragma unroll
+      for (int j = 0; j < G; ++j)
+#pragma unroll
+        for (int e = 0; e < EPL; ++e)
+          ll_put(pbase + j * (HD + 2) + lane * EPL + e, fw[j] * acc[j][e], tag_out);
+    }
+    if (tid < G) {
+      float mx = -INFINITY, ls = 0.f;
+      for (int w = 0; w < NCW; ++w) mx = fmaxf(mx, att_ml[(w * G + tid) * 2]);
+      for (int w = 0; w < NCW; ++w) {
+        const float lw = att_ml[(w * G + tid) * 2 + 1];
+        if (lw > 0.f) ls += lw * expf(att_ml[(w * G + tid) * 2] - mx);
+      }
+      ll_put(pbase + tid * (HD + 2) + HD, mx, tag_out);
+      ll_put(pbase + tid * (HD + 2) + HD + 1, ls, tag_out);
+    }
+  }
+  // release the kept slot once every warp is done with it
+  if (keep_slot >= 0) {
+    named_sync(1, NCT);
+    if (lane == 0) mbar_arrive(&t->empty[keep_slot]);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Merge the attention partials of all S splits for elements [e0, e0 + kb) of
+// the concatenated head outputs (nq * hd) into ov (shared memory), in a fixed
+// split order: o_e = sum_s exp(m_s - m) acc_s[e] / sum_s exp(m_s - m) l_s,
+// per q head.  Scratch in uni: staged values [0, MERGE_STAGE), then (m, l)
+// and weights of every split for each head the block touches.
+// ----------------------------------------------------------------------------
+template <int HD, int GQ>
+__device__ __forceinline__ bool att_merge_block(const DevModel& M, int S, int e0, int kb,
+                                                float* uni, float* ov, uint32_t tag,
+                                                SmemTail* t, int* err, long long wait_ns,
+                                                int tid) {
+  const int h_lo = e0 / HD, nhb = (e0 + kb - 1) / HD - h_lo + 1;
+  float* stage = uni;
+  float* mls = uni + MERGE_STAGE;        // [S][nhb][2]
+  float* wgt = mls + 2 * S * nhb;        // [S][nhb]
+  // address of element c (< HD: accumulator, HD: m, HD + 1: l) of q head hq, split si
+  auto part = [&](int si, int hq, int c) {
+    return M.part_ll + ((size_t(hq / GQ) * kMaxCtas + si) * GQ + hq % GQ) * (HD + 2) + c;
+  };
+  // (m, l) of every split for the block's heads
+  if (!poll_words<per_thread(MERGE_ML_MAX)>(
+          mls, S * nhb * 2,
+          [&](int w) { return part(w / (nhb * 2), h_lo + (w >> 1) % nhb, HD + (w & 1)); }, tag, t,
+          err, wait_ns, tid))
+    return false;
+  if (tid < nhb) {
+    float mx = -INFINITY;
+    for (int si = 0; si < S; ++si) mx = fmaxf(mx, mls[(si * nhb + tid) * 2]);
+    float den = 0.f;
+    for (int si = 0; si < S; ++si) {
+      const float f = expf(mls[(si * nhb + tid) * 2] - mx);
+      wgt[si * nhb + tid] = f;
+      den = fmaf(f, mls[(si * nhb + tid) * 2 + 1], den);
+    }
+    const float inv = 1.0f / den;
+    for (int si = 0; si < S; ++si) wgt[si * nhb + tid] *= inv;
+  }
+  for (int e = tid; e < kb; e += NCT) ov[e] = 0.f;
+  named_sync(1, NCT);
+  // accumulator values, a batch of splits at a time
+  const int sb_max = MERGE_STAGE / kb;
+  for (int s0 = 0; s0 < S; s0 += sb_max) {
+    const int sb = min(sb_max, S - s0);
+    if (!poll_words<per_thread(MERGE_STAGE)>(
+            stage, sb * kb,
+            [&](int w) {
+              const int e = e0 + w % kb;
+              return part(s0 + w / kb, e / HD, e % HD);
+            },
+            tag, t, err, wait_ns, tid))
+      return false;
+    for (int e = tid; e < kb; e += NCT) {
+      const int hb = (e0 + e) / HD - h_lo;
+      float o = ov[e];
+      for (int q = 0; q < sb; ++q) o = fmaf(wgt[(s0 + q) * nhb + hb], stage[q * kb + e], o);
+      ov[e] = o;
     }
     named_sync(1, NCT);
   }
-  // publish this split's partial as tagged words: per head [acc(HD) | m | l]
-  unsigned long long* part = M.part_ll + size_t(gidx) * kMaxCtas * G * (HD + 2);
-  unsigned long long* pbase = part + size_t(d.unit_s) * G * (HD + 2);
-  for (int i = tid; i < G * HD; i += NCT) ll_put(pbase + (i / HD) * (HD + 2) + (i % HD), att_acc[i], tag_out);
-  if (tid < G) {
-    float mx = -INFINITY, ls = 0.f;
-    for (int w = 0; w < NCW; ++w) mx = fmaxf(mx, att_ml[(w * G + tid) * 2]);
-    for (int w = 0; w < NCW; ++w) {
-      const float lw = att_ml[(w * G + tid) * 2 + 1];
-      if (lw > 0.f) ls += lw * expf(att_ml[(w * G + tid) * 2] - mx);
-    }
-    ll_put(pbase + tid * (HD + 2) + HD, mx, tag_out);
-    ll_put(pbase + tid * (HD + 2) + HD + 1, ls, tag_out);
-  }
-  // Cooperative merge: every split CTA of the group merges its slice
-  // [e0, e1) of the group's G*HD outputs from all S partials.  The (m, l)
-  // words of all splits double as the group's completion signal.
-  const int S = d.S;
-  const int e0 = (G * HD) * d.unit_s / S, e1 = (G * HD) * (d.unit_s + 1) / S;
-  const int ne = e1 - e0;
-  constexpr int ATT_SCRATCH = 2 * G * HD + 2 * HD + NCW * G * 2;
-  float* mls = uni + ATT_SCRATCH;  // [S][G][2]  (m, l) of every split
-  float* wgt = mls + S * G * 2;    // [S][G]     merge weights
-  float* stage = uni;              // [S][ne]    the slice's partial values (att_q is free now)
-  bool ok2 = true;
-  {
-    uint64_t start = 0;
-    for (int it = 0;; ++it) {
-      bool stale = false;
-#pragma unroll 4
-      for (int w = tid; w < S * G * 2; w += NCT) {
-        const int si = w / (G * 2), j = (w >> 1) % G, c = w & 1;
-        const unsigned long long v = ll_get(part + (size_t(si) * G + j) * (HD + 2) + HD + c);
-        if (uint32_t(v >> 32) != tag_out) stale = true;
-        else mls[w] = __uint_as_float(uint32_t(v));
-      }
-      if (!stale) break;
-      if (it == 0) start = global_ns();
-      else if ((it & 7) == 0 && give_up(t, M.err, start, a.wait_ns)) { ok2 = false; break; }
-    }
-  }
-  if (named_sync_or(1, NCT, !ok2)) return;
-  if (tid < G) {
-    float mx = -INFINITY;
-    for (int si = 0; si < S; ++si) mx = fmaxf(mx, mls[(si * G + tid) * 2]);
-    float den = 0.f;
-    for (int si = 0; si < S; ++si) {
-      const float f = expf(mls[(si * G + tid) * 2] - mx);
-      wgt[si * G + tid] = f;
-      den = fmaf(f, mls[(si * G + tid) * 2 + 1], den);
-    }
-    const float inv = 1.0f / den;
-    for (int si = 0; si < S; ++si) wgt[si * G + tid] *= inv;
-  }
-  {
-    uint64_t start = 0;
-    for (int it = 0;; ++it) {
-      bool stale = false;
-#pragma unroll 4
-      for (int w = tid; w < S * ne; w += NCT) {
-        const int si = w / ne, e = e0 + w % ne;
-        const unsigned long long v = ll_get(part + (size_t(si) * G + e / HD) * (HD + 2) + e % HD);
-        if (uint32_t(v >> 32) != tag_out) stale = true;
-        else stage[w] = __uint_as_float(uint32_t(v));
-      }
-      if (!stale) break;
-      if (it == 0) start = global_ns();
-      else if ((it & 7) == 0 && give_up(t, M.err, start, a.wait_ns)) { ok2 = false; break; }
-    }
-  }
-  if (named_sync_or(1, NCT, !ok2)) return;
-  for (int w = tid; w < ne; w += NCT) {
-    const int e = e0 + w, j = e / HD;
-    float o = 0.f;
-    for (int si = 0; si < S; ++si) o = fmaf(wgt[si * G + j], stage[si * ne + w], o);
-    ll_put(M.atto_ll + size_t(gidx) * G * HD + e, o, tag_out);
-  }
+  return true;
 }
 
 // ----------------------------------------------------------------------------
@@ -989,58 +1296,37 @@ __device__ __forceinline__ void attention_phase(const DevModel& M, const StepArg
 constexpr size_t PF_AHEAD = size_t(64) << 10;  // L2 prefetch distance per CTA (bytes)
 
 struct ChunkCursor {
-  int l, p, np, gp;
-  int kinds[8];
-  PD d;
+  const PD* tab;
+  int np;     // phases in the launch
+  int gp;     // current phase
   int r;      // first row of the current chunk
   bool done;
-  __device__ __forceinline__ int nrows() const { return min(d.rpc, d.r0 + d.n - r); }
-  __device__ __forceinline__ uint32_t bytes() const { return uint32_t(nrows()) * d.row_bytes; }
-  __device__ __forceinline__ const char* src0() const { return d.p0 + size_t(r) * d.row_bytes; }
-  __device__ __forceinline__ const char* src1() const { return d.p1 + size_t(r) * d.row_bytes; }
+  __device__ __forceinline__ const PD& d() const { return tab[gp]; }
+  __device__ __forceinline__ int nrows() const { return min(d().rpc, d().r0 + d().n - r); }
+  __device__ __forceinline__ uint32_t bytes() const { return uint32_t(nrows()) * d().row_bytes; }
+  __device__ __forceinline__ const char* src0() const { return d().p0 + size_t(r) * d().row_bytes; }
+  __device__ __forceinline__ const char* src1() const { return d().p1 + size_t(r) * d().row_bytes; }
 };
 
-// Move to the first chunk at or after phase (l, p); skips empty phases.
-__device__ __noinline__ void cursor_settle(ChunkCursor& c, const DevModel& M,
-                                              const StepArgs& a, int cta, uint64_t pol_w,
-                                              uint64_t pol_s) {
-  while (true) {
-    if (c.l > M.n_layers) {
-      c.done = true;
-      return;
-    }
-    if (c.p >= c.np) {
-      ++c.l;
-      c.p = 0;
-      if (c.l < M.n_layers) c.np = layer_phases(M.layers[c.l], c.kinds);
-      else if (c.l == M.n_layers) { c.kinds[0] = PH_LM; c.np = 1; }
-      continue;
-    }
-    c.d = describe(M, a, c.kinds[c.p], c.l < M.n_layers ? c.l : 0, c.gp, cta, pol_w, pol_s);
-    c.r = c.d.r0;
-    if (c.d.n > 0) return;
-    ++c.p;
-    ++c.gp;
-  }
+// Move to the first chunk at or after phase gp; skips empty phases.
+__device__ __forceinline__ void cursor_settle(ChunkCursor& c) {
+  while (c.gp < c.np && c.tab[c.gp].n == 0) ++c.gp;
+  c.done = c.gp >= c.np;
+  if (!c.done) c.r = c.tab[c.gp].r0;
 }
 
-__device__ __forceinline__ void cursor_init(ChunkCursor& c, const DevModel& M, const StepArgs& a,
-                                            int cta, uint64_t pol_w, uint64_t pol_s) {
-  c.l = 0;
-  c.p = 0;
+__device__ __forceinline__ void cursor_init(ChunkCursor& c, const PD* tab, int np) {
+  c.tab = tab;
+  c.np = np;
   c.gp = 0;
-  c.done = false;
-  c.np = layer_phases(M.layers[0], c.kinds);
-  cursor_settle(c, M, a, cta, pol_w, pol_s);
+  cursor_settle(c);
 }
 
-__device__ __forceinline__ void cursor_next(ChunkCursor& c, const DevModel& M, const StepArgs& a,
-                                            int cta, uint64_t pol_w, uint64_t pol_s) {
-  c.r += c.d.rpc;
-  if (c.r < c.d.r0 + c.d.n) return;
-  ++c.p;
+__device__ __forceinline__ void cursor_next(ChunkCursor& c) {
+  c.r += c.d().rpc;
+  if (c.r < c.d().r0 + c.d().n) return;
   ++c.gp;
-  cursor_settle(c, M, a, cta, pol_w, pol_s);
+  cursor_settle(c);
 }
 
 // ----------------------------------------------------------------------------
@@ -1052,7 +1338,8 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
   unsigned char* ring = smem_raw;
   SmemTail* t = reinterpret_cast<SmemTail*>(smem_raw + size_t(NSLOT) * SLOT);
   float* uni = reinterpret_cast<float*>(smem_raw + size_t(NSLOT) * SLOT + sizeof(SmemTail));
-  float* xraw = uni + UNION_FLOATS;
+  float* xraw = uni + UNION_FLOATS;  // the residual stream (identical in every CTA)
+  PD* tab = reinterpret_cast<PD*>(xraw + XRAW_MAX);  // this CTA's schedule, one entry per phase
 
   const DevModel& M = a.m;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1071,6 +1358,13 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
     t->token = tok;
     fence_barrier_init();
   }
+  // The schedule: this CTA's share of every phase, one phase per thread.
+  const int n_phases = M.n_layers * PHASES_PER_LAYER + 1;
+  for (int i = tid; i < n_phases; i += NTHR) {
+    int l;
+    const int kind = phase_kind(M, i, l);
+    tab[i] = describe(M, a, kind, l, i, cta);
+  }
   // RoPE table for this position (angles in double: pos * theta^(-2i/hd)).
   for (int i = tid; i < HD / 2; i += NTHR) {
     double inv_freq = pow(double(M.theta), -2.0 * double(i) / double(HD));
@@ -1078,6 +1372,15 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
     sincos(double(a.pos) * inv_freq, &s, &c);
     t->rope_cos[i] = float(c);
     t->rope_sin[i] = float(s);
+  }
+  // Clear this CTA's share of the other launch parity's sum words: the next
+  // launch adds into them (this launch adds into its own parity's words,
+  // cleared by the launch before it or by mk_reset).
+  const size_t xacc_words = size_t(M.n_layers) * 2 * M.H;
+  {
+    unsigned long long* other = M.xacc + size_t((a.seq & 1u) ^ 1u) * xacc_words;
+    const size_t z0 = xacc_words * cta / M.ncta, z1 = xacc_words * (cta + 1) / M.ncta;
+    for (size_t i = z0 + tid; i < z1; i += NTHR) other[i] = 0ull;
   }
   __syncthreads();
 
@@ -1093,8 +1396,8 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
   if (warp == NCW) {
     if (lane != 0) return;
     ChunkCursor ld, pf;
-    cursor_init(ld, M, a, cta, pol_w, pol_s);
-    cursor_init(pf, M, a, cta, pol_w, pol_s);
+    cursor_init(ld, tab, n_phases);
+    cursor_init(pf, tab, n_phases);
     size_t ld_bytes = 0, pf_bytes = 0;
     uint32_t g = 0;
     while (!ld.done && !aborted(t)) {
@@ -1102,22 +1405,24 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
       while (!pf.done && pf_bytes < ld_bytes + PF_AHEAD) {
         const uint32_t b = pf.bytes();
         bulk_prefetch_l2(pf.src0(), b);
-        if (pf.d.p1) bulk_prefetch_l2(pf.src1(), b);
-        pf_bytes += size_t(b) * (pf.d.p1 ? 2 : 1);
-        cursor_next(pf, M, a, cta, pol_w, pol_s);
+        if (pf.d().p1) bulk_prefetch_l2(pf.src1(), b);
+        pf_bytes += size_t(b) * (pf.d().p1 ? 2 : 1);
+        cursor_next(pf);
       }
       const int slot = int(g % NSLOT);
       if (g >= NSLOT && !bounded_wait(&t->empty[slot], ((g / NSLOT) - 1) & 1, t, M.err, a.wait_ns))
         break;
       const uint32_t bytes = ld.bytes();
       unsigned char* dst = ring + size_t(slot) * SLOT;
-      mbar_arrive_expect_tx(&t->full[slot], bytes * (ld.d.p1 ? 2u : 1u));
-      bulk_g2s(dst, ld.src0(), bytes, &t->full[slot], ld.d.pol);
-      if (ld.d.p1)
-        bulk_g2s(dst + size_t(ld.d.rpc) * ld.d.row_bytes, ld.src1(), bytes, &t->full[slot], ld.d.pol);
-      ld_bytes += size_t(bytes) * (ld.d.p1 ? 2 : 1);
+      const PD& ldd = ld.d();
+      const uint64_t pol = ldd.keep ? pol_s : pol_w;
+      mbar_arrive_expect_tx(&t->full[slot], bytes * (ldd.p1 ? 2u : 1u));
+      bulk_g2s(dst, ld.src0(), bytes, &t->full[slot], pol);
+      if (ldd.p1)
+        bulk_g2s(dst + size_t(ldd.rpc) * ldd.row_bytes, ld.src1(), bytes, &t->full[slot], pol);
+      ld_bytes += size_t(bytes) * (ldd.p1 ? 2 : 1);
       ++g;
-      cursor_next(ld, M, a, cta, pol_w, pol_s);
+      cursor_next(ld);
     }
     // Let every copy still in flight land before the CTA may exit.
     const uint32_t first = g > uint32_t(NSLOT) ? g - NSLOT : 0u;
@@ -1132,14 +1437,20 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
 
   // ======================= consumer warps ===================================
   const int tok = t->token;
-  const uint16_t* emb_row = M.embed + size_t(tok) * M.H;
+  const int grp = group_of(M, cta);
+  unsigned long long* xacc = M.xacc + size_t(a.seq & 1u) * xacc_words;  // [n_layers][2][H]
   uint32_t g = 0;  // chunk counter (same order as the producer)
   int gp = 0;
   int kinds[8];
-  // tags of the latest producer of each tagged buffer
-  uint32_t tag_x = 0, tag_inp = 0, tag_dno = 0, tag_qkv = 0, tag_att = 0,
-           tag_h = 0;
-  int xb = 0;  // residual buffer holding the latest x
+  uint32_t tag_qkv = 0, tag_att = 0;  // producers of the attention exchanges
+  uint32_t tag_inp = 0, tag_h = 0;    // producers of the group exchanges
+  float* ovec = uni + UNION_FLOATS - 256;  // merged attention block (<= 256 floats)
+
+  // the residual stream starts as the token's embedding row (every CTA)
+  {
+    const uint16_t* emb_row = M.embed + size_t(tok) * M.H;
+    for (int i = tid; i < M.H; i += NCT) xraw[i] = bf2f(emb_row[i]);
+  }
 
   for (int l = 0; l <= M.n_layers; ++l) {
     const bool lm = (l == M.n_layers);
@@ -1150,60 +1461,102 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
 
     for (int p = 0; p < np; ++p, ++gp) {
       const int kind = kinds[p];
-      const PD d = describe(M, a, kind, lm ? 0 : l, gp, cta, pol_w, pol_s);
+      const PD d = tab[gp];
       const uint32_t tag_me = make_tag(a.seq, gp);
-      // debug hook: the inputs of phase `fail_phase` carry a tag nobody writes
-      const uint32_t dbg = gp == a.fail_phase ? 0x80000000u : 0u;
+      // debug hook: the inputs of phase `fail_phase` can never complete
+      const bool fail_here = gp == a.fail_phase;
+      const uint32_t dbg = fail_here ? 0x80000000u : 0u;
+      const int want = M.ng + (fail_here ? 1 : 0);
       // uniform across the consumer warps (also orders the previous phase)
       const bool dry = named_sync_or(1, NCT, aborted(t));
       GemvJob j{};  // matrix phases fill it in; one dispatch after the switch
       j.d = d;
       j.tag = tag_me;
+      j.err = M.err;
+      j.scale = 1.f;
       bool gemv = false;
+      const float* xs = uni;
       switch (kind) {
         case PH_DN_IN:
         case PH_QKV:
         case PH_GU:
         case PH_LM: {
-          // input: RMSNorm of the residual stream (the embedding at layer 0)
+          // input: the residual stream completed by the previous split-K sum
+          // (none before layer 0), then its RMSNorm
           bool ok = true;
           // union layout in this phase: x [0, 2048) | conv history [2048, 3072)
           // (<= CONV_ROWS_MAX float4) | conv taps [3072, 3584) (<= CONV_ROWS_MAX uint2)
           float4* conv_s = reinterpret_cast<float4*>(uni + 2048);
           uint2* conv_taps = reinterpret_cast<uint2*>(uni + 2048 + 4 * CONV_ROWS_MAX);
-          float4* conv_g = reinterpret_cast<float4*>(M.conv_state[a.st_buf]) + size_t(L.sub) * M.ch;
           const uint16_t* gain = kind == PH_GU ? L.mlp_norm
                                  : kind == PH_LM ? M.final_norm : L.attn_norm;
           float gv[GK];
           load_gains(gv, gain, M.H, tid);
+          float ss = 0.f;
+          const int src_layer = kind == PH_GU ? l : l - 1;
+          const int src_half = kind == PH_GU ? 0 : 1;
           if (!dry) {
-            if (kind == PH_DN_IN) {
+            if (kind == PH_DN_IN && grp >= 0) {
               // stage the conv history and taps of this CTA's q|k|v rows first
               // (independent of the input: their latency overlaps the wait)
-              const int nconv = max(0, min(d.r0 + d.n, M.ch) - d.r0);
+              const int nconv = max(0, min(d.r0 + d.n, 2 * M.dk + M.dv) - d.r0);
+              const float4* conv_in =
+                  reinterpret_cast<const float4*>(M.conv_state[a.st_in]) + size_t(L.sub) * M.ch;
+              GemvJob cj{};
+              cj.dk = M.dk;
+              cj.chan_q = grp * M.dk;
+              cj.chan_k = M.nh * M.dk + grp * M.dk;
+              cj.chan_v = 2 * M.nh * M.dk + grp * M.dv;
               for (int i = tid; i < nconv; i += NCT) {
-                conv_s[i] = conv_g[d.r0 + i];
-                conv_taps[i] = *reinterpret_cast<const uint2*>(L.conv_w + size_t(d.r0 + i) * 4);
+                const int ch = conv_channel(cj, d.r0 + i);
+                conv_s[i] = conv_in[ch];
+                conv_taps[i] = *reinterpret_cast<const uint2*>(L.conv_w + size_t(ch) * 4);
               }
             }
-            if (l == 0 && kind != PH_GU) {
-              for (int i = tid; i < M.H; i += NCT) uni[i] = bf2f(emb_row[i]);
+            // the residual stream (completed by the split-K sum) and x * gain,
+            // the RMSNorm numerator; the GEMV scales its results by the norm
+            if (src_layer >= 0) {
+              ss = cfa_read_add<GK>(xraw, uni, gv,
+                                    xacc + (size_t(src_layer) * 2 + src_half) * M.H, M.H, want,
+                                    t, M.err, a.wait_ns, tid, ok);
             } else {
-              ok = ll_gather<per_thread(XRAW_MAX)>(uni, M.x_ll + size_t(xb) * M.H, M.H,
-                                                   tag_x | dbg, t, M.err, a.wait_ns, tid);
+#pragma unroll
+              for (int k = 0; k < GK; ++k) {
+                const int i = tid + k * NCT;
+                if (i < M.H) {
+                  const float v = xraw[i];
+                  uni[i] = v * gv[k];
+                  ss = fmaf(v, v, ss);
+                }
+              }
             }
           }
+          ss = warp_sum(ss);
+          if (lane == 0) t->red[warp] = ss;
           const bool bad = named_sync_or(1, NCT, !ok);
-          if (!dry && !bad)
-            rmsnorm_inplace(uni, kind == PH_LM ? nullptr : xraw, gv, M.H, M.eps, t, tid);
+          if (!dry && !bad) {
+            if (src_half == 1 && src_layer >= 0 && cta == 0 && a.hidden)
+              for (int i = tid; i < M.H; i += NCT) a.hidden[size_t(src_layer) * M.H + i] = xraw[i];
+            float tot = 0.f;
+#pragma unroll
+            for (int w = 0; w < NCW; ++w) tot += t->red[w];
+            j.scale = 1.0f / sqrtf(tot / float(M.H) + M.eps);
+          }
           gemv = true;
           if (kind == PH_DN_IN) {
             j.epi = EPI_INPROJ;
-            j.dst = M.inp_ll;
+            j.dst = M.grp_inp + size_t(grp < 0 ? 0 : grp) * M.rin_h;
             j.conv_s = conv_s;
             j.conv_taps = conv_taps;
-            j.conv_out = conv_g;
-            j.ch = M.ch;
+            j.conv_out = reinterpret_cast<float4*>(M.conv_state[a.st_out]) + size_t(L.sub) * M.ch;
+            j.dk = M.dk;
+            j.nconv = 2 * M.dk + M.dv;
+            j.chan_q = grp * M.dk;
+            j.chan_k = M.nh * M.dk + grp * M.dk;
+            j.chan_v = 2 * M.nh * M.dk + grp * M.dv;
+            j.row_b = 2 * M.dk + 2 * M.dv;
+            j.a_log = grp >= 0 ? L.A_log[grp] : 0.f;
+            j.dt_bias = grp >= 0 ? L.dt_bias[grp] : 0.f;
             tag_inp = tag_me;
           } else if (kind == PH_QKV) {
             j.epi = EPI_STORE;
@@ -1211,7 +1564,8 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
             tag_qkv = tag_me;
           } else if (kind == PH_GU) {
             j.epi = EPI_SWIGLU;
-            j.dst = M.mlph_ll;
+            j.dst = M.grp_h + size_t(grp < 0 ? 0 : grp) * M.kb_mlp;
+            j.dst_off = (grp < 0 ? 0 : grp) * M.kb_mlp;
             tag_h = tag_me;
           } else {
             j.epi = EPI_LOGITS;
@@ -1219,85 +1573,55 @@ __global__ void __launch_bounds__(NTHR, 1) decode_kernel(const __grid_constant__
           }
           break;
         }
-        case PH_OUT: {
-          bool ok = true;
-          const int K = L.is_attn ? M.nq * M.hd : M.nh * M.dv;
-          constexpr int EPL_G = DK / 32;  // gated-norm elements per lane (dv == dk)
-          float gw[EPL_G];
-#pragma unroll
-          for (int e = 0; e < EPL_G; ++e) gw[e] = L.is_attn ? 0.f : bf2f(L.out_norm[lane * EPL_G + e]);
-          if (!dry) {
-            if (L.is_attn) {
-              ok = ll_gather<per_thread(UNION_FLOATS)>(uni, M.atto_ll, K, tag_att | dbg, t, M.err,
-                                                       a.wait_ns, tid);
-            } else {
-              // gated RMSNorm of the readout: o_h from the state phase, z_h
-              // from the in-projection (z staged in the upper half of uni)
-              // o (tagged by the state phase) and z (by the in-projection)
-              // in one polling round
-              const LLSeg sg[2] = {{M.dno_ll, uni, K, tag_dno | dbg},
-                                   {M.inp_ll + M.ch, uni + 2048, K, tag_inp}};
-              ok = ll_gather_segs<per_thread(4096), 2>(sg, t, M.err, a.wait_ns, tid);
-            }
-          }
-          const bool bad = named_sync_or(1, NCT, !ok);
-          if (!dry && !bad && !L.is_attn) {
-            constexpr int EPL = DK / 32;  // dv == dk
-            for (int h = warp; h < M.nh; h += NCW) {
-              float o[EPL];
-              float ss = 0.f;
-#pragma unroll
-              for (int e = 0; e < EPL; ++e) {
-                o[e] = uni[h * DK + lane * EPL + e];
-                ss = fmaf(o[e], o[e], ss);
-              }
-              ss = warp_sum(ss);
-              const float inv = 1.0f / sqrtf(ss / float(DK) + M.eps);
-#pragma unroll
-              for (int e = 0; e < EPL; ++e) {
-                const int i = lane * EPL + e;
-                uni[h * DK + i] = o[e] * inv * gw[e] * siluf_(uni[2048 + h * DK + i]);
-              }
-            }
-            named_sync(1, NCT);
-          }
-          gemv = true;
-          j.epi = EPI_RESID;
-          j.dst = M.x_ll + size_t(xb ^ 1) * M.H;
-          j.xraw = xraw;
-          xb ^= 1;
-          tag_x = tag_me;
-          break;
-        }
-        case PH_DOWN: {
-          bool ok = true;
-          if (!dry)
-            ok = ll_gather<per_thread(UNION_FLOATS)>(uni, M.mlph_ll, M.I, tag_h | dbg, t, M.err,
-                                                     a.wait_ns, tid);
-          named_sync_or(1, NCT, !ok);
-          gemv = true;
-          j.epi = EPI_RESID;
-          j.dst = M.x_ll + size_t(xb ^ 1) * M.H;
-          j.xraw = xraw;
-          j.hidden = a.hidden ? a.hidden + size_t(l) * M.H : nullptr;
-          xb ^= 1;
-          tag_x = tag_me;
-          break;
-        }
         case PH_DN_ST:
-          dn_state_phase<DK>(M, a, L, d, g, ring, t, uni, tag_inp | dbg, tag_me, dry, tid, warp,
+          dn_state_phase<DK>(M, a, L, d, g, ring, t, uni, tag_inp | dbg, dry, grp, tid, warp,
                              lane);
-          tag_dno = tag_me;
+          break;
+        case PH_DN_OUTP:
+          // the head's gated output (left in uni + 2048 + DK by the state
+          // phase) times the head's K block of the output projection
+          gemv = true;
+          xs = uni + 2048 + DK;
+          j.epi = EPI_CFA;
+          j.dst = xacc + (size_t(l) * 2 + 0) * M.H;
           break;
         case PH_ATT:
-          attention_phase<HD, GQ>(M, a, L, d, g, ring, t, uni, tag_qkv, dbg, tag_me,
-                                  dry, tid, warp, lane);
+          attention_phase<HD, GQ>(M, a, L, d, g, ring, t, uni, tag_qkv, dbg, tag_me, dry, tid,
+                                  warp, lane);
           tag_att = tag_me;
           break;
+        case PH_ATT_OUTP: {
+          bool ok = true;
+          if (!dry && grp >= 0)
+            ok = att_merge_block<HD, GQ>(M, att_splits(M, a.pos), grp * M.kb_att, M.kb_att, uni,
+                                         ovec, tag_att | dbg, t, M.err, a.wait_ns, tid);
+          named_sync_or(1, NCT, !ok);
+          gemv = true;
+          xs = ovec;
+          j.epi = EPI_CFA;
+          j.dst = xacc + (size_t(l) * 2 + 0) * M.H;
+          break;
+        }
+        case PH_DOWNP: {
+          // the group's K block of SiLU(gate)*up, then the down-projection partial
+          bool ok = true;
+          if (!dry && grp >= 0)
+            ok = ll_gather<per_thread(UNION_FLOATS)>(uni, M.grp_h + size_t(grp) * M.kb_mlp,
+                                                     M.kb_mlp, tag_h | dbg, t, M.err, a.wait_ns,
+                                                     tid);
+          named_sync_or(1, NCT, !ok);
+          gemv = true;
+          j.epi = EPI_CFA;
+          j.dst = xacc + (size_t(l) * 2 + 1) * M.H;
+          break;
+        }
         default:
           break;
       }
-      if (gemv) g = gemv_core(j, g, ring, t, M.err, a.wait_ns, uni);
+      if (gemv)
+        g = (j.epi == EPI_CFA && d.row_bytes <= 1024)
+                ? gemv_short(j, g, ring, t, M.err, a.wait_ns, xs)
+                : gemv_core(j, g, ring, t, M.err, a.wait_ns, xs);
     }
   }
 

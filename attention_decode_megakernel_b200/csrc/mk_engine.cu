@@ -8,6 +8,7 @@
 #include <new>
 
 #include "mk.h"
+#include "mk_chunk.cuh"
 #include "mk_decode.cuh"
 #include "mk_delta.cuh"
 #include "mk_model.cuh"
@@ -23,11 +24,16 @@ struct Layout {
   size_t model;
   size_t dn_state[mk::kStateBufs], conv_state[mk::kStateBufs];
   size_t kc, vc;
-  size_t x, inp, dno, qkv, atto, mlph, part, hidden, logits, tickets, err, amax;
-  size_t wqkv;  // packed q|k|v weight rows of every attention layer
+  size_t xacc, grp_inp, grp_h, qkv, part, hidden, logits, tickets, err, amax;
+  // weight copies laid out for the decode kernel's groups
+  size_t wqkv;      // q|k|v rows of every attention layer
+  size_t w_in_pk;   // DeltaNet in-projection rows per head
+  size_t w_out_blk; // output projections by K block
+  size_t w_down_blk;  // MLP down projections by K block
   // multi-token prompt path: T_MAX positions per chunk
   int tmax, pw, aw;
   size_t pf_tok, pf_x, pf_xn, pf_p, pf_c, pf_o, pf_a16, pf_qk, pf_bak, pf_att, pf_part;
+  size_t pf_chunk;  // chunkwise delta rule operands: [nh][chunks][block]
   size_t total;
 };
 
@@ -64,7 +70,6 @@ Layout make_layout(const mk_config& c) {
   const int n_attn = count_attn(c), n_dn = c.n_layers - n_attn;
   const size_t ch = size_t(2) * c.dn_heads * c.dn_dk + size_t(c.dn_heads) * c.dn_dv;
   const size_t rin = ch + size_t(c.dn_heads) * c.dn_dv + 2 * size_t(c.dn_heads);
-  const size_t M = size_t(c.max_verify);
   const size_t G = size_t(c.q_heads / c.kv_heads);
   L.model = take(sizeof(DevModel));
   for (int b = 0; b < mk::kStateBufs; ++b) {
@@ -75,13 +80,20 @@ Layout make_layout(const mk_config& c) {
   L.kc = take(kv);
   L.vc = take(kv);
   L.wqkv = take(size_t(n_attn) * (c.q_heads + 2 * c.kv_heads) * c.head_dim * c.hidden * 2);
-  L.x = take(2 * M * c.hidden * 8);
-  L.inp = take(M * rin * 8);
-  L.dno = take(M * c.dn_heads * c.dn_dv * 8);
-  L.qkv = take(M * size_t(c.q_heads + 2 * c.kv_heads) * c.head_dim * 8);
-  L.atto = take(M * size_t(c.q_heads) * c.head_dim * 8);
-  L.mlph = take(M * size_t(c.mlp) * 8);
-  L.part = take(size_t(c.kv_heads) * mk::kMaxCtas * M * G * (c.head_dim + 2) * 8);
+  const size_t rin_h = 2 * size_t(c.dn_dk) + 2 * size_t(c.dn_dv) + 2;
+  L.w_in_pk = take(size_t(n_dn) * c.dn_heads * rin_h * c.hidden * 2);
+  {
+    size_t outw = 0;  // K of every layer's output projection
+    for (int l = 0; l < c.n_layers; ++l)
+      outw += c.layer_is_attn[l] ? size_t(c.q_heads) * c.head_dim : size_t(c.dn_heads) * c.dn_dv;
+    L.w_out_blk = take(outw * c.hidden * 2);
+  }
+  L.w_down_blk = take(size_t(c.n_layers) * c.hidden * c.mlp * 2);
+  L.xacc = take(size_t(2) * c.n_layers * 2 * c.hidden * 8);
+  L.grp_inp = take(size_t(c.dn_heads) * rin_h * 8);
+  L.grp_h = take(size_t(c.mlp + c.dn_heads) * 8);
+  L.qkv = take(size_t(c.q_heads + 2 * c.kv_heads) * c.head_dim * 8);
+  L.part = take(size_t(c.kv_heads) * mk::kMaxCtas * G * (c.head_dim + 2) * 8);
   L.hidden = take(size_t(c.n_layers) * c.hidden * 4);
   L.logits = take(size_t(c.vocab) * 4);
   L.tickets = take(4);
@@ -114,6 +126,8 @@ Layout make_layout(const mk_config& c) {
     // split-K partial sums of a prompt GEMM with few output tiles (< 100):
     // k_split x T x n_out <= (148 + tiles) x 128 x 128 floats
     L.pf_part = take(size_t(kSplitPartialTiles) * mk::pf::BM * mk::pf::BN * 4);
+    const size_t blk = c.dn_dk == 64 ? mk::ck::Blk<64>::FLOATS : mk::ck::Blk<128>::FLOATS;
+    L.pf_chunk = take(size_t(c.dn_heads) * ((T + mk::ck::C - 1) / mk::ck::C) * blk * 4);
   }
   L.total = off;
   return L;
@@ -229,8 +243,8 @@ int read_device_error(mk_engine* e) {
   return err;
 }
 
-int launch_decode(mk_engine* e, int pos, int st_buf, int token, int tok_src, float* logits,
-                  int32_t* tok_out) {
+int launch_decode(mk_engine* e, int pos, int st_in, int st_out, int token, int tok_src,
+                  float* logits, int32_t* tok_out) {
   mk::StepArgs a;
   a.m = e->hm;
   a.pos = pos;
@@ -238,15 +252,18 @@ int launch_decode(mk_engine* e, int pos, int st_buf, int token, int tok_src, flo
   a.tok_src = tok_src;
   a.amax_in = e->amax_toggle;
   a.amax_out = e->amax_toggle ^ 1;
-  a.st_buf = st_buf;
+  a.st_in = st_in;
+  a.st_out = st_out;
   a.logits = logits ? logits : reinterpret_cast<float*>(e->ws + e->lay.logits);
   a.tok_out = tok_out;
   a.hidden = reinterpret_cast<float*>(e->ws + e->lay.hidden);
-  e->seq = e->seq + 1 >= (1u << 23) ? 1u : e->seq + 1;
-  a.seq = e->seq;
+  // the sequence number names the launch in exchange tags, and its parity
+  // selects the set of split-K sum words (consecutive launches alternate)
+  uint32_t seq = e->seq + 1;
+  if (seq >= (1u << 23)) seq = (seq & 1u) ? 1u : 2u;
+  a.seq = seq;
   a.fail_phase = e->fail_phase;
   a.wait_ns = e->wait_ns;
-  e->fail_phase = -1;
   void* args[] = {&a};
   cudaError_t err = cudaLaunchCooperativeKernel(e->var->fn, dim3(e->ncta), dim3(mk::NTHR), args,
                                                 e->var->smem, e->stream);
@@ -254,10 +271,24 @@ int launch_decode(mk_engine* e, int pos, int st_buf, int token, int tok_src, flo
     cudaGetLastError();
     return MK_ERR_LAUNCH;
   }
+  e->seq = seq;
+  e->fail_phase = -1;
   e->amax_toggle ^= 1;
   e->amax_valid = true;
   e->launches += 1;
   return MK_OK;
+}
+
+// One decode launch at the current position that advances the state: it
+// reads the current state buffer and writes the next one in the ring.
+int decode_advance(mk_engine* e, int token, int tok_src, float* logits, int32_t* tok_out) {
+  const int nxt = (e->cur_buf + 1) % mk::kStateBufs;
+  const int rc = launch_decode(e, e->pos, e->cur_buf, nxt, token, tok_src, logits, tok_out);
+  if (rc == MK_OK) {
+    e->cur_buf = nxt;
+    e->pos += 1;
+  }
+  return rc;
 }
 
 // One tensor-core GEMM launch.  For a chunk of at most one token tile with
@@ -375,18 +406,29 @@ int run_chunk(mk_engine* e, const int32_t* tokens_host, int T, const int* ck_buf
       float* S = m.dn_state[e->cur_buf] + size_t(D.sub) * nh * dv * dk;
       const dim3 rgrid(nh, dv / (REC_WARPS * REC_RPW));
       const int vcol = 2 * nh * dk;
-      if (dk == 128 && ck_bufs)
+      if (!ck_bufs) {
+        // prompt chunk: the chunkwise-parallel form (independent per
+        // chunk of 64 positions, then one pass over the chunks)
+        float* prep = reinterpret_cast<float*>(ws + L.pf_chunk);
+        const dim3 pg((T + mk::ck::C - 1) / mk::ck::C, nh), sg(dv / mk::ck::SCAN_ROWS, nh);
+        if (dk == 128) {
+          mk::ck::chunk_prep_kernel<128><<<pg, mk::ck::PREP_THREADS, mk::ck::prep_smem<128>(), st>>>(
+              QK, BAK, Cv + vcol, size_t(m.ch), size_t(dk), T, prep);
+          mk::ck::chunk_scan_kernel<128><<<sg, mk::ck::SCAN_THREADS, mk::ck::scan_smem<128>(), st>>>(
+              S, prep, T, O, size_t(nh) * dv, size_t(dv));
+        } else {
+          mk::ck::chunk_prep_kernel<64><<<pg, mk::ck::PREP_THREADS, mk::ck::prep_smem<64>(), st>>>(
+              QK, BAK, Cv + vcol, size_t(m.ch), size_t(dk), T, prep);
+          mk::ck::chunk_scan_kernel<64><<<sg, mk::ck::SCAN_THREADS, mk::ck::scan_smem<64>(), st>>>(
+              S, prep, T, O, size_t(nh) * dv, size_t(dv));
+        }
+        e->launches += 1;  // two kernels where the scan was one
+      } else if (dk == 128 && ck_bufs)
         recurrence_kernel<128, true><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, Cv, m.ch, vcol,
                                                                        O, nh * dv, T, cks);
-      else if (dk == 128)
-        recurrence_kernel<128, false><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, Cv, m.ch, vcol,
-                                                                        O, nh * dv, T, cks);
-      else if (ck_bufs)
+      else
         recurrence_kernel<64, true><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, Cv, m.ch, vcol,
                                                                       O, nh * dv, T, cks);
-      else
-        recurrence_kernel<64, false><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, Cv, m.ch, vcol,
-                                                                       O, nh * dv, T, cks);
       gated_norm_kernel<<<dim3(T, nh), dv, 0, st>>>(O, nh * dv, P, pw, m.ch, D.out_norm, A16, aw,
                                                     c.rms_eps, lo_a);
       if (rc == MK_OK) rc = launch_gemm(e, mp.out, e->map_a16_dn, X, H, H, T, nh * dv, 1);
@@ -511,13 +553,36 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
   cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
   if (!coop || nsm <= 0) return MK_ERR_LAUNCH;
   const int ncta = nsm < mk::kMaxCtas ? nsm : mk::kMaxCtas;
+  // the decode kernel keeps its per-launch schedule in shared memory
+  if (c.n_layers * mk::PHASES_PER_LAYER + 1 > mk::MAX_PHASES) return MK_ERR_UNSUPPORTED;
+  // decode groups: one per DeltaNet head, gs CTAs each
+  const int ng = c.dn_heads, gs = ncta / ng;
+  if (gs < 1 || ng > 255) return MK_ERR_UNSUPPORTED;
+  if ((c.q_heads * c.head_dim) % ng || c.mlp % ng) return MK_ERR_UNSUPPORTED;
+  const int kb_att = c.q_heads * c.head_dim / ng, kb_mlp = c.mlp / ng;
+  const int rin_h = 2 * c.dn_dk + 2 * c.dn_dv + 2;
+  // K blocks of the split-K rows: 16-byte rows; the attention block fits
+  // the merge staging; the conv staging holds a CTA's in-projection rows
+  if (kb_att % 8 || kb_mlp % 8 || kb_att > 256 || kb_att > mk::MERGE_STAGE)
+    return MK_ERR_UNSUPPORTED;
+  if ((rin_h + gs - 1) / gs > mk::CONV_ROWS_MAX) return MK_ERR_UNSUPPORTED;
   {
-    // attention merge scratch: (m, l) and weights of every split
+    // attention scratch of the split phase, and of the merge: staged values,
+    // (m, l) and weights of every split for the q heads one block touches
     const int smax = ncta / c.kv_heads;
     const int att = 2 * G * c.head_dim + 2 * c.head_dim + mk::NCW * G * 2;
-    if (att + smax * G * 3 > mk::UNION_FLOATS || G * c.head_dim + smax > att)
+    const int nhb = (kb_att + c.head_dim - 1) / c.head_dim + 1;
+    if (att > mk::UNION_FLOATS || nhb > mk::MERGE_HEADS_MAX ||
+        2 * smax * nhb > mk::MERGE_ML_MAX ||
+        mk::MERGE_STAGE + 3 * smax * nhb > mk::UNION_FLOATS - 256)
       return MK_ERR_UNSUPPORTED;
   }
+  // the kernel's balanced splits multiply in 32 bits
+  if (uint64_t(c.max_ctx + 1) * ncta >= (uint64_t(1) << 32) ||
+      uint64_t(c.vocab) * ncta >= (uint64_t(1) << 32))
+    return MK_ERR_UNSUPPORTED;
+  // one DeltaNet head's state is one ring chunk of the state phase
+  if (size_t(c.dn_dv) * c.dn_dk * 4 > size_t(mk::SLOT)) return MK_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(var->fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            int(var->smem)) != cudaSuccess) {
     cudaGetLastError();
@@ -530,17 +595,6 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
     cudaGetLastError();
     return MK_ERR_LAUNCH;
   }
-  // the DeltaNet head cache, row values and conv staging must fit a CTA's
-  // shared scratch
-  if ((2 * c.dn_heads * c.dn_dk + 2 * c.dn_heads * c.dn_dv + 2 * c.dn_heads + ncta - 1) / ncta >
-      mk::CONV_ROWS_MAX)
-    return MK_ERR_UNSUPPORTED;
-  {
-    int rows = (c.dn_heads * c.dn_dv + ncta - 1) / ncta;
-    int heads = rows / c.dn_dv + 2;
-    if (heads > mk::DN_HEADS_MAX || rows > mk::DN_ROWS_MAX) return MK_ERR_UNSUPPORTED;
-  }
-
   mk_engine* e = new (std::nothrow) mk_engine();
   if (!e) return MK_ERR_ARG;
   e->cfg = c;
@@ -573,6 +627,11 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
   m.max_ctx = c.max_ctx;
   m.max_verify = c.max_verify;
   m.ncta = ncta;
+  m.ng = ng;
+  m.gs = gs;
+  m.rin_h = rin_h;
+  m.kb_att = kb_att;
+  m.kb_mlp = kb_mlp;
   m.eps = c.rms_eps;
   m.theta = c.rope_theta;
   m.embed = static_cast<const uint16_t*>(w->embed);
@@ -593,6 +652,9 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
     D.w_v = static_cast<const uint16_t*>(L.w_v);
     D.w_o = static_cast<const uint16_t*>(L.w_o);
     D.w_qkv = nullptr;
+    D.w_in_pk = nullptr;
+    D.w_out_blk = nullptr;
+    D.w_down_blk = nullptr;
     D.mlp_norm = static_cast<const uint16_t*>(L.mlp_norm);
     D.w_gate = static_cast<const uint16_t*>(L.w_gate);
     D.w_up = static_cast<const uint16_t*>(L.w_up);
@@ -608,33 +670,73 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
   m.kc = reinterpret_cast<uint16_t*>(ws + lay.kc);
   m.vc = reinterpret_cast<uint16_t*>(ws + lay.vc);
   {
-    // the decode kernel reads each attention layer's q, k and v rows as one
-    // matrix: pack them once into the workspace
+    // Weight copies for the decode kernel's partition (made once, on the
+    // engine's stream): each attention layer's q, k and v rows as one
+    // matrix; each DeltaNet head's in-projection rows q|k|v|z|b|a
+    // contiguous; every output projection and MLP down projection split into
+    // ng blocks of K columns, block g stored as its own [H][K/ng] matrix.
+    cudaStream_t st = e->stream;
+    cudaError_t r = cudaSuccess;
     const size_t H2 = size_t(c.hidden) * 2;
     const size_t qb = size_t(c.q_heads) * c.head_dim * H2, kb = size_t(c.kv_heads) * c.head_dim * H2;
-    for (int l = 0; l < c.n_layers; ++l) {
+    const size_t dkr = size_t(c.dn_dk) * H2, dvr = size_t(c.dn_dv) * H2;
+    char* out_dst = ws + lay.w_out_blk;
+    for (int l = 0; l < c.n_layers && r == cudaSuccess; ++l) {
       mk::DevLayer& D = m.layers[l];
-      if (!D.is_attn) continue;
-      char* dst = ws + lay.wqkv + size_t(D.sub) * (qb + 2 * kb);
-      cudaError_t r = cudaMemcpyAsync(dst, D.w_q, qb, cudaMemcpyDeviceToDevice, e->stream);
-      if (r == cudaSuccess)
-        r = cudaMemcpyAsync(dst + qb, D.w_k, kb, cudaMemcpyDeviceToDevice, e->stream);
-      if (r == cudaSuccess)
-        r = cudaMemcpyAsync(dst + qb + kb, D.w_v, kb, cudaMemcpyDeviceToDevice, e->stream);
-      if (r != cudaSuccess) {
-        delete e;
-        return cuda_status(r);
+      // split-K copy of a [H][K] matrix into ng blocks [H][K/ng]
+      auto blocks = [&](char* dst, const void* src, int K) {
+        const size_t kbytes = size_t(K / ng) * 2;
+        for (int g = 0; g < ng && r == cudaSuccess; ++g)
+          r = cudaMemcpy2DAsync(dst + size_t(g) * c.hidden * kbytes, kbytes,
+                                static_cast<const char*>(src) + size_t(g) * kbytes, size_t(K) * 2,
+                                kbytes, size_t(c.hidden), cudaMemcpyDeviceToDevice, st);
+      };
+      if (D.is_attn) {
+        char* dst = ws + lay.wqkv + size_t(D.sub) * (qb + 2 * kb);
+        r = cudaMemcpyAsync(dst, D.w_q, qb, cudaMemcpyDeviceToDevice, st);
+        if (r == cudaSuccess) r = cudaMemcpyAsync(dst + qb, D.w_k, kb, cudaMemcpyDeviceToDevice, st);
+        if (r == cudaSuccess)
+          r = cudaMemcpyAsync(dst + qb + kb, D.w_v, kb, cudaMemcpyDeviceToDevice, st);
+        D.w_qkv = reinterpret_cast<const uint16_t*>(dst);
+        blocks(out_dst, D.w_o, c.q_heads * c.head_dim);
+        D.w_out_blk = reinterpret_cast<const uint16_t*>(out_dst);
+        out_dst += size_t(c.q_heads) * c.head_dim * H2;
+      } else {
+        const char* src = reinterpret_cast<const char*>(D.in_proj);
+        char* dst = ws + lay.w_in_pk + size_t(D.sub) * c.dn_heads * rin_h * H2;
+        D.w_in_pk = reinterpret_cast<const uint16_t*>(dst);
+        const size_t ch_rows = 2 * size_t(c.dn_heads) * c.dn_dk + size_t(c.dn_heads) * c.dn_dv;
+        for (int h = 0; h < c.dn_heads && r == cudaSuccess; ++h) {
+          // rows of head h in the caller's layout [q | k | v | z | b | a]
+          const size_t seg_src[6] = {
+              size_t(h) * dkr, size_t(c.dn_heads) * dkr + h * dkr,
+              2 * size_t(c.dn_heads) * dkr + h * dvr, ch_rows * H2 + h * dvr,
+              (ch_rows + size_t(c.dn_heads) * c.dn_dv + h) * H2,
+              (ch_rows + size_t(c.dn_heads) * c.dn_dv + c.dn_heads + h) * H2};
+          const size_t seg_len[6] = {dkr, dkr, dvr, dvr, H2, H2};
+          for (int q = 0; q < 6 && r == cudaSuccess; ++q) {
+            r = cudaMemcpyAsync(dst, src + seg_src[q], seg_len[q], cudaMemcpyDeviceToDevice, st);
+            dst += seg_len[q];
+          }
+        }
+        blocks(out_dst, D.out_proj, c.dn_heads * c.dn_dv);
+        D.w_out_blk = reinterpret_cast<const uint16_t*>(out_dst);
+        out_dst += size_t(c.dn_heads) * c.dn_dv * H2;
       }
-      D.w_qkv = reinterpret_cast<const uint16_t*>(dst);
+      char* ddst = ws + lay.w_down_blk + size_t(l) * c.mlp * H2;
+      blocks(ddst, D.w_down, c.mlp);
+      D.w_down_blk = reinterpret_cast<const uint16_t*>(ddst);
+    }
+    if (r != cudaSuccess) {
+      delete e;
+      return cuda_status(r);
     }
   }
   using ull = unsigned long long;
-  m.x_ll = reinterpret_cast<ull*>(ws + lay.x);
-  m.inp_ll = reinterpret_cast<ull*>(ws + lay.inp);
-  m.dno_ll = reinterpret_cast<ull*>(ws + lay.dno);
+  m.xacc = reinterpret_cast<ull*>(ws + lay.xacc);
+  m.grp_inp = reinterpret_cast<ull*>(ws + lay.grp_inp);
+  m.grp_h = reinterpret_cast<ull*>(ws + lay.grp_h);
   m.qkv_ll = reinterpret_cast<ull*>(ws + lay.qkv);
-  m.atto_ll = reinterpret_cast<ull*>(ws + lay.atto);
-  m.mlph_ll = reinterpret_cast<ull*>(ws + lay.mlph);
   m.part_ll = reinterpret_cast<ull*>(ws + lay.part);
   m.hidden = reinterpret_cast<float*>(ws + lay.hidden);
   m.logits_scratch = reinterpret_cast<float*>(ws + lay.logits);
@@ -649,7 +751,19 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
     return MK_ERR_CUDA;
   }
   // tensor maps of the prompt path (weights and the chunk's bf16 activations)
-  e->pf_ok = cudaFuncSetAttribute(mk::pf::gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e->pf_ok = cudaFuncSetAttribute(mk::ck::chunk_prep_kernel<128>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(mk::ck::prep_smem<128>())) == cudaSuccess &&
+             cudaFuncSetAttribute(mk::ck::chunk_scan_kernel<128>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(mk::ck::scan_smem<128>())) == cudaSuccess &&
+             cudaFuncSetAttribute(mk::ck::chunk_prep_kernel<64>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(mk::ck::prep_smem<64>())) == cudaSuccess &&
+             cudaFuncSetAttribute(mk::ck::chunk_scan_kernel<64>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(mk::ck::scan_smem<64>())) == cudaSuccess &&
+             cudaFuncSetAttribute(mk::pf::gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   int(mk::pf::GEMM_SMEM)) == cudaSuccess &&
              cudaFuncSetAttribute(mk::pf::gemm_tc_partial,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -706,7 +820,7 @@ int mk_reset(mk_engine* e) {
                           (b + 1 < mk::kStateBufs ? L.dn_state[b + 1] : L.kc) - L.conv_state[b],
                           e->stream);
   }
-  if (r == cudaSuccess) r = cudaMemsetAsync(e->ws + L.x, 0, L.total - L.x, e->stream);
+  if (r == cudaSuccess) r = cudaMemsetAsync(e->ws + L.xacc, 0, L.total - L.xacc, e->stream);
   if (r != cudaSuccess) return cuda_status(r);
   e->pos = 0;
   e->cur_buf = 0;
@@ -731,9 +845,7 @@ int mk_decode_step(mk_engine* e, int32_t token, float* logits_out) {
   if (token < 0 || token >= e->cfg.vocab) return MK_ERR_ARG;
   if (e->pending_verify) return MK_ERR_STATE;
   if (e->pos + 1 > e->cfg.max_ctx) return MK_ERR_CTX_OVERFLOW;
-  int rc = launch_decode(e, e->pos, e->cur_buf, token, 0, logits_out, nullptr);
-  if (rc == MK_OK) e->pos += 1;
-  return rc;
+  return decode_advance(e, token, 0, logits_out, nullptr);
 }
 
 int mk_generate(mk_engine* e, int32_t first_token, int n, int32_t* tokens_out,
@@ -746,10 +858,8 @@ int mk_generate(mk_engine* e, int32_t first_token, int n, int32_t* tokens_out,
   for (int i = 0; i < n; ++i) {
     float* lg = logits_out ? logits_out + size_t(i) * e->cfg.vocab : nullptr;
     const int from_device = (i > 0 || first_token == -1) ? 1 : 0;
-    int rc = launch_decode(e, e->pos, e->cur_buf, first_token < 0 ? 0 : first_token, from_device,
-                           lg, tokens_out + i);
+    int rc = decode_advance(e, first_token < 0 ? 0 : first_token, from_device, lg, tokens_out + i);
     if (rc != MK_OK) return rc;
-    e->pos += 1;
   }
   return MK_OK;
 }
@@ -772,10 +882,8 @@ int mk_prefill(mk_engine* e, const int32_t* tokens_host, int n, float* logits_ou
   }
   // the rest (at least the last position: its logits and greedy argmax)
   for (; i < n; ++i) {
-    int rc = launch_decode(e, e->pos, e->cur_buf, tokens_host[i], 0,
-                           i == n - 1 ? logits_out : nullptr, nullptr);
+    int rc = decode_advance(e, tokens_host[i], 0, i == n - 1 ? logits_out : nullptr, nullptr);
     if (rc != MK_OK) return rc;
-    e->pos += 1;
   }
   return MK_OK;
 }
@@ -796,20 +904,13 @@ int mk_verify(mk_engine* e, const int32_t* tokens_host, int n, float* logits_out
     e->amax_valid = false;
     return MK_OK;
   }
-  const Layout& L = e->lay;
-  const size_t dn_bytes = L.conv_state[0] - L.dn_state[0];
-  const size_t conv_bytes = (mk::kStateBufs > 1 ? L.dn_state[1] : L.kc) - L.conv_state[0];
+  // no chunk path: one decode launch per position, each reading the state
+  // after the previous position and writing its own checkpoint buffer
   int src = e->cur_buf, k = 0;
   for (int j = 0; j < n; ++j) {
-    int dst = (e->cur_buf + 1 + j) % mk::kStateBufs;
+    const int dst = (e->cur_buf + 1 + j) % mk::kStateBufs;
     e->verify_bufs[j] = dst;
-    cudaError_t r = cudaMemcpyAsync(e->ws + L.dn_state[dst], e->ws + L.dn_state[src], dn_bytes,
-                                    cudaMemcpyDeviceToDevice, e->stream);
-    if (r == cudaSuccess)
-      r = cudaMemcpyAsync(e->ws + L.conv_state[dst], e->ws + L.conv_state[src], conv_bytes,
-                          cudaMemcpyDeviceToDevice, e->stream);
-    if (r != cudaSuccess) return cuda_status(r);
-    int rc = launch_decode(e, e->pos + j, dst, tokens_host[j], 0,
+    int rc = launch_decode(e, e->pos + j, src, dst, tokens_host[j], 0,
                            logits_out + size_t(j) * e->cfg.vocab, nullptr);
     if (rc != MK_OK) return rc;
     src = dst;
@@ -932,6 +1033,73 @@ int mk_delta_step(float* S, const void* q, const void* k, const void* v, const f
   return cuda_status(cudaGetLastError());
 }
 
+size_t mk_delta_chunked_ws_bytes(int T, int heads, int dk) {
+  if (T <= 0 || heads <= 0 || (dk != 64 && dk != 128)) return 0;
+  const size_t nc = (size_t(T) + mk::ck::C - 1) / mk::ck::C;
+  const size_t blk = dk == 64 ? mk::ck::Blk<64>::FLOATS : mk::ck::Blk<128>::FLOATS;
+  return align256(size_t(heads) * T * 2 * dk * 4) + align256(size_t(heads) * T * 16) +
+         size_t(heads) * nc * blk * 4;
+}
+
+int mk_delta_chunked(float* S, const float* q, const float* k, const float* v,
+                     const float* alpha, const float* beta, float* o, int T, int heads, int dk,
+                     int dv, void* workspace, size_t ws_bytes, void* stream) {
+  if (!S || !q || !k || !v || !alpha || !beta || !o || !workspace || T <= 0 || heads <= 0)
+    return MK_ERR_ARG;
+  if (dk != dv || (dk != 64 && dk != 128)) return MK_ERR_UNSUPPORTED;
+  if (!aligned16(S) || !aligned16(workspace) || ws_bytes < mk_delta_chunked_ws_bytes(T, heads, dk))
+    return MK_ERR_ARG;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return MK_ERR_CUDA;
+  }
+  if (!attr_done[dev]) {
+    if (cudaFuncSetAttribute(mk::ck::chunk_prep_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(mk::ck::prep_smem<128>())) != cudaSuccess ||
+        cudaFuncSetAttribute(mk::ck::chunk_scan_kernel<128>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(mk::ck::scan_smem<128>())) != cudaSuccess ||
+        cudaFuncSetAttribute(mk::ck::chunk_prep_kernel<64>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(mk::ck::prep_smem<64>())) != cudaSuccess ||
+        cudaFuncSetAttribute(mk::ck::chunk_scan_kernel<64>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(mk::ck::scan_smem<64>())) != cudaSuccess) {
+      cudaGetLastError();
+      return MK_ERR_CUDA;
+    }
+    attr_done[dev] = true;
+  }
+  char* ws = static_cast<char*>(workspace);
+  float* QK = reinterpret_cast<float*>(ws);
+  float4* BAK = reinterpret_cast<float4*>(ws + align256(size_t(heads) * T * 2 * dk * 4));
+  float* prep = reinterpret_cast<float*>(ws + align256(size_t(heads) * T * 2 * dk * 4) +
+                                         align256(size_t(heads) * T * 16));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t n_pos = size_t(heads) * T;
+  const int pb = int((n_pos * dk + 255) / 256 < 4096 ? (n_pos * dk + 255) / 256 : 4096);
+  const dim3 pg((T + mk::ck::C - 1) / mk::ck::C, heads), sg(dv / mk::ck::SCAN_ROWS, heads);
+  // v and o are [heads][T][dv]: position stride dv, head stride T * dv
+  const size_t ts = size_t(dv), hs = size_t(T) * dv;
+  if (dk == 128) {
+    mk::ck::chunk_pack_kernel<128><<<pb, 256, 0, st>>>(q, k, alpha, beta, n_pos, QK, BAK);
+    mk::ck::chunk_prep_kernel<128><<<pg, mk::ck::PREP_THREADS, mk::ck::prep_smem<128>(), st>>>(
+        QK, BAK, v, ts, hs, T, prep);
+    mk::ck::chunk_scan_kernel<128><<<sg, mk::ck::SCAN_THREADS, mk::ck::scan_smem<128>(), st>>>(
+        S, prep, T, o, ts, hs);
+  } else {
+    mk::ck::chunk_pack_kernel<64><<<pb, 256, 0, st>>>(q, k, alpha, beta, n_pos, QK, BAK);
+    mk::ck::chunk_prep_kernel<64><<<pg, mk::ck::PREP_THREADS, mk::ck::prep_smem<64>(), st>>>(
+        QK, BAK, v, ts, hs, T, prep);
+    mk::ck::chunk_scan_kernel<64><<<sg, mk::ck::SCAN_THREADS, mk::ck::scan_smem<64>(), st>>>(
+        S, prep, T, o, ts, hs);
+  }
+  return cuda_status(cudaGetLastError());
+}
+
 int mk_debug_gemm(const void* W, const void* X, float* C, int n_out, int T, int K,
                   void* stream) {
   if (!W || !X || !C || n_out <= 0 || T <= 0 || K <= 0 || K % 64) return MK_ERR_ARG;
@@ -961,9 +1129,16 @@ int mk_debug_gemm(const void* W, const void* X, float* C, int n_out, int T, int 
   g.k_split = 1;
   g.err = err_word;
   g.wait_ns = 2000000000LL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the error word starts each call at zero (stream-ordered); a tile that
+  // gives up sets it and C is then filled with NaN
+  const cudaError_t mr = cudaMemsetAsync(err_word, 0, 4, st);
+  if (mr != cudaSuccess) return cuda_status(mr);
   const dim3 grid((n_out + mk::pf::BM - 1) / mk::pf::BM, (T + mk::pf::BN - 1) / mk::pf::BN);
-  mk::pf::gemm_tc<<<grid, mk::pf::GEMM_THREADS, mk::pf::GEMM_SMEM,
-                    static_cast<cudaStream_t>(stream)>>>(g);
+  mk::pf::gemm_tc<<<grid, mk::pf::GEMM_THREADS, mk::pf::GEMM_SMEM, st>>>(g);
+  const size_t n = size_t(T) * n_out;
+  mk::pf::poison_on_error_kernel<<<int((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256, 0,
+                                   st>>>(err_word, n, C);
   return cuda_status(cudaGetLastError());
 }
 
@@ -972,7 +1147,7 @@ int mk_debug_gemm(const void* W, const void* X, float* C, int n_out, int T, int 
 namespace {
 // Static device scratch of the allocation-free GEMM entry point: split-K
 // partial sums (at most kNoAllocFloats floats = 8 MiB) and its wait-error
-// word (zero when the module loads; written only when a wait runs out).
+// word (cleared at the start of every call; set when a wait runs out).
 constexpr size_t kNoAllocFloats = size_t(2) << 20;
 __device__ __align__(256) float g_noalloc_partial[kNoAllocFloats];
 __device__ __align__(256) int g_noalloc_err;
@@ -1031,12 +1206,17 @@ int mk_debug_gemm_noalloc(const void* W, const void* X, float* C, int n_out, int
   g.err = g_err_addr[dev];
   g.wait_ns = 2000000000LL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the error word starts each call at zero (stream-ordered, no allocation);
+  // a range that gives up sets it and the reduction then writes NaN
+  const cudaError_t mr = cudaMemsetAsync(g_err_addr[dev], 0, 4, st);
+  if (mr != cudaSuccess) return cuda_status(mr);
   const dim3 grid((n_out + mk::pf::BM - 1) / mk::pf::BM, (T + mk::pf::BN - 1) / mk::pf::BN, ks);
   mk::pf::gemm_tc_partial<<<grid, mk::pf::GEMM_THREADS, mk::pf::GEMM_SMEM, st>>>(
       g, g_partial_addr[dev]);
   const size_t n = size_t(T) * n_out;
   const int rblocks = int((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-  mk::pf::splitk_reduce_kernel<<<rblocks, 256, 0, st>>>(g_partial_addr[dev], ks, n, C);
+  mk::pf::splitk_reduce_kernel<<<rblocks, 256, 0, st>>>(g_partial_addr[dev], ks, n, C,
+                                                        g_err_addr[dev]);
   return cuda_status(cudaGetLastError());
 }
 
@@ -1050,6 +1230,7 @@ const char* mk_strerror(int s) {
     case MK_ERR_TIMEOUT: return "device-side wait gave up";
     case MK_ERR_CUDA: return "CUDA runtime error";
     case MK_ERR_UNSUPPORTED: return "shape not implemented by the kernels";
+    case MK_ERR_RANGE: return "decode partial sum outside the fixed-point range";
     default: return "unknown status";
   }
 }

@@ -17,8 +17,12 @@ struct DevLayer {
   const float *A_log, *dt_bias;
   const uint16_t *out_norm, *out_proj;
   const uint16_t *w_q, *w_k, *w_v, *w_o;
-  const uint16_t* w_qkv;  // engine copy of q|k|v rows, [(nq + 2 nkv) hd][H]
   const uint16_t *mlp_norm, *w_gate, *w_up, *w_down;
+  // engine copies laid out for the decode kernel's group partition
+  const uint16_t* w_qkv;       // attention q|k|v rows, [(nq + 2 nkv) hd][H]
+  const uint16_t* w_in_pk;     // DeltaNet in-proj rows per head, [nh][q|k|v|z|b|a][H]
+  const uint16_t* w_out_blk;   // output projection by K block, [ng][H][K / ng]
+  const uint16_t* w_down_blk;  // MLP down projection by K block, [ng][H][I / ng]
   int is_attn;
   int sub;  // index among layers of the same kind
 };
@@ -30,6 +34,8 @@ struct DevModel {
   int nh, dk, dv, ck, ch, rin;      // DeltaNet: heads, dims, conv taps/channels, in_proj rows
   int nq, nkv, hd;                  // attention
   int max_ctx, max_verify, ncta;
+  int ng, gs;                       // decode groups (one per DeltaNet head) and CTAs per group
+  int rin_h, kb_att, kb_mlp;        // in-proj rows per head; K block of the attention / MLP partials
   float eps, theta;
   // weights
   const uint16_t *embed, *final_norm;
@@ -38,15 +44,13 @@ struct DevModel {
   float *dn_state[kStateBufs];      // [n_dn][nh][dv][dk]
   float *conv_state[kStateBufs];    // [n_dn][ch][4]  (3 taps of history + pad)
   uint16_t *kc, *vc;                // [n_attn][nkv][max_ctx][hd]
-  // activations exchanged between CTAs, as tagged words {fp32 value, tag}
-  // (M = max_verify rows where noted)
-  unsigned long long *x_ll;     // [2][M][H]  residual stream (double-buffered)
-  unsigned long long *inp_ll;   // [M][rin]   in-proj output: conv'd q|k|v, raw z|b|a
-  unsigned long long *dno_ll;   // [M][nh*dv] DeltaNet readout o = S q
-  unsigned long long *qkv_ll;   // [M][(nq+2nkv)*hd] raw attention projections
-  unsigned long long *atto_ll;  // [M][nq*hd] attention output (merged)
-  unsigned long long *mlph_ll;  // [M][I]     SiLU(gate)*up
-  unsigned long long *part_ll;  // [nkv][kMaxCtas][M*group][hd+2] split-K attention partials (tagged)
+  // decode exchange buffers: tagged words {fp32 value, tag} and count-carrying
+  // fixed-point sums (see mk_decode.cuh)
+  unsigned long long *xacc;     // [2 launch parities][n_layers][2][H] residual deltas
+  unsigned long long *grp_inp;  // [ng][rin_h] one head's in-projection outputs
+  unsigned long long *grp_h;    // [ng][I / ng] one group's SiLU(gate)*up values
+  unsigned long long *qkv_ll;   // [(nq+2nkv)*hd] raw attention projections
+  unsigned long long *part_ll;  // [nkv][kMaxCtas][group][hd+2] split-K attention partials
   float *hidden;   // [n_layers][H] residual after each layer (last position)
   float *logits_scratch;  // [V]
   unsigned *tickets;      // [1] grid argmax ticket

@@ -270,14 +270,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 }
 
 // C[t][n] = sum over z of partial[z][t][n], in order z = 0, 1, ... (a split-K
-// result that does not depend on the order the ranges finished in).
-__global__ void splitk_reduce_kernel(const float* partial, int k_split, size_t n, float* c) {
+// result that does not depend on the order the ranges finished in).  When
+// the GEMM's wait-error word is set (a tile gave up and left its partial
+// unwritten) every element of C becomes NaN instead.
+__global__ void splitk_reduce_kernel(const float* partial, int k_split, size_t n, float* c,
+                                     const int* err) {
+  const bool failed = err && *reinterpret_cast<const volatile int*>(err) != 0;
   for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += size_t(gridDim.x) * blockDim.x) {
     float acc = 0.f;
     for (int z = 0; z < k_split; ++z) acc += partial[size_t(z) * n + i];
-    c[i] = acc;
+    c[i] = failed ? __int_as_float(0x7FC00000) : acc;
   }
+}
+
+// C becomes NaN when the GEMM's wait-error word is set (a tile gave up and
+// left its part of C unwritten).
+__global__ void poison_on_error_kernel(const int* err, size_t n, float* c) {
+  if (*reinterpret_cast<const volatile int*>(err) == 0) return;
+  for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += size_t(gridDim.x) * blockDim.x)
+    c[i] = __int_as_float(0x7FC00000);
 }
 
 // c[t][n] (+)= sum over z of partial[z][t][n] (z = 0, 1, ... in order), for

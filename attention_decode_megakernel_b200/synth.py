@@ -234,6 +234,32 @@ def make_delta_sweep(B: int, steps: int, heads: int = 16, dk: int = 128,
     return {"S0": S0, "q": q, "k": k, "v": v, "beta": beta, "alpha": alpha}
 
 
+def make_delta_sequence(heads: int, T: int, dk: int = 128, alpha_lo: float = 0.3,
+                        seed: int = SEED_SWEEP + 10) -> Dict:
+    """Inputs of a whole-sequence gated delta rule (the prompt path's shape:
+    one sequence, `heads` heads, T positions), all float32.
+
+    S0 ~ N(0, 0.1^2) [heads][dk][dk]; q, k ~ N(0,1) scaled to unit length
+    (input preparation, float64) [heads][T][dk]; v ~ N(0,1) [heads][T][dk];
+    beta ~ U(0,1), alpha ~ U(alpha_lo, 1) [heads][T] (the 0.8B-shaped
+    model's random weights give alpha near 0.5).
+    """
+    rng = np.random.default_rng(seed)
+    S0 = rng.standard_normal((heads, dk, dk), dtype=np.float32) * np.float32(0.1)
+
+    def unit_rows(shape):
+        z = rng.standard_normal(shape, dtype=np.float32).astype(np.float64)
+        z /= np.sqrt((z * z).sum(axis=-1, keepdims=True))
+        return z.astype(np.float32)
+
+    q = unit_rows((heads, T, dk))
+    k = unit_rows((heads, T, dk))
+    v = rng.standard_normal((heads, T, dk), dtype=np.float32)
+    beta = rng.uniform(0.0, 1.0, size=(heads, T)).astype(np.float32)
+    alpha = rng.uniform(alpha_lo, 1.0, size=(heads, T)).astype(np.float32)
+    return {"S0": S0, "q": q, "k": k, "v": v, "beta": beta, "alpha": alpha}
+
+
 # --------------------------------------------------------------------------
 # synthetic engine state (long-context and verify parity without a long
 # prompt through the oracle)

@@ -47,16 +47,21 @@ typedef enum {
   MK_ERR_LAUNCH = 4,       /* cooperative launch impossible / failed        */
   MK_ERR_TIMEOUT = 5,      /* a device-side wait gave up (error word set)   */
   MK_ERR_CUDA = 6,         /* another CUDA runtime error                    */
-  MK_ERR_UNSUPPORTED = 7   /* shape outside what the kernels implement      */
+  MK_ERR_UNSUPPORTED = 7,  /* shape outside what the kernels implement      */
+  MK_ERR_RANGE = 8         /* a decode partial sum left the fixed-point range
+                              of the split-K reduction (|value| >= 8192)     */
 } mk_status;
 
 /* Model shape.  Layer l is full attention when layer_is_attn[l] != 0 and a
  * Gated-DeltaNet layer otherwise.  Shapes the decode kernel is built for:
  * hidden % 256 == 0 and <= 2048; conv_k == 4; mlp % 8 == 0 and <= 4096; the embedding
  * tied to the LM head; q_heads == 4 * kv_heads; and (dn_dk == dn_dv,
- * head_dim) one of (64, 64), (128, 128), (128, 256).  mk_create returns
- * MK_ERR_UNSUPPORTED otherwise (also when a CTA's share of a phase exceeds
- * the kernel's shared-memory staging). */
+ * head_dim) one of (64, 64), (128, 128), (128, 256); mlp and
+ * q_heads * head_dim divisible by dn_heads (the decode groups' K blocks,
+ * each a multiple of 8 and the attention block at most 256 wide); at least
+ * one SM per DeltaNet head.  mk_create returns MK_ERR_UNSUPPORTED otherwise
+ * (also when a CTA's share of a phase exceeds the kernel's shared-memory
+ * staging). */
 typedef struct {
   int32_t n_layers;
   uint8_t layer_is_attn[MK_MAX_LAYERS];
@@ -100,21 +105,27 @@ typedef struct {
 typedef struct mk_engine mk_engine;
 
 /* Bytes of device workspace mk_create needs for this config (recurrent
- * state, verify checkpoints, KV cache, activations, exchange words, and a
- * packed copy of each attention layer's q|k|v weight rows).
+ * state, verify checkpoints, KV cache, activations, exchange words, and the
+ * decode kernel's copies of the layer weights, see mk_create).
  * Returns 0 for an invalid config. */
 size_t mk_workspace_bytes(const mk_config *cfg);
 
-/* Create an engine on the current CUDA device.  `workspace` (device, at
+/* Create an engine on the current CUDA device for the hybrid stack of the
+ * launch post "OS Megakernel that match M5 Max Tok/w at 2x the Throughput on
+ * RTX 3090" (kernel bullet list: the whole forward pass of one token in one
+ * dispatch).  `workspace` (device, at
  * least mk_workspace_bytes(cfg) bytes, 256-byte aligned) and the weights
  * stay owned by the caller and must outlive the engine; the engine only
  * keeps pointers.  `cuda_stream` (a cudaStream_t, may be NULL for the
  * legacy stream) is the stream every later call runs on.  Checks that one
  * CTA of the decode kernel fits on every SM (cooperative co-residency) and
- * returns MK_ERR_LAUNCH otherwise.  Copies each attention layer's w_q, w_k
- * and w_v into one [q|k|v][hidden] block of the workspace (the decode
- * kernel reads them as one matrix), so later changes to those three weights
- * need a new engine.  Zeroes the state (as mk_reset). */
+ * returns MK_ERR_LAUNCH otherwise.  Copies weights into the workspace in
+ * the layouts the decode kernel's CTA groups read (one group per DeltaNet
+ * head): each attention layer's w_q, w_k and w_v as one [q|k|v][hidden]
+ * matrix, each DeltaNet head's in_proj rows (q|k|v|z|b|a of that head) as
+ * one block, and every out_proj, w_o and w_down split into dn_heads column
+ * blocks; later changes to the caller's weights need a new engine.  Zeroes
+ * the state (as mk_reset). */
 int mk_create(const mk_config *cfg, const mk_weights *w, void *workspace,
               size_t ws_bytes, void *cuda_stream, mk_engine **out);
 
@@ -122,7 +133,10 @@ int mk_create(const mk_config *cfg, const mk_weights *w, void *workspace,
 void mk_destroy(mk_engine *e);
 
 /* Zero the DeltaNet and conv states, empty the KV cache, clear a device
- * error and any pending verify.  Weights are untouched. */
+ * error and any pending verify: the start of a new sequence (launch post,
+ * "Why nobody had done this yet?": the DeltaNet layers carry a recurrent
+ * state and the attention layers a KV cache from token to token).  Weights
+ * are untouched. */
 int mk_reset(mk_engine *e);
 
 /* Run n prompt tokens (host array, values in [0, vocab)) through the stack
@@ -169,7 +183,10 @@ int mk_generate(mk_engine *e, int32_t first_token, int n, int32_t *tokens_out,
 
 /* Verify n tokens at once (1 <= n <= max_verify), the speculative-decoding
  * shape (several draft tokens checked by one forward pass, with the
- * recurrent state checkpointed for rollback): the stack runs over positions
+ * recurrent state checkpointed for rollback; the follow-up post
+ * "업데이트: 단일 RTX 3090에서 Qwen 3.8 27B를 140 tok/s로 구동 (Megakernel:
+ * KL divergence", speed list: four draft tokens checked for the cost of one
+ * forward pass, greedy output unchanged): the stack runs over positions
  * pos .. pos+n-1 as one chunk -- every projection one tensor-core GEMM with
  * M = n (weights read once for the n positions), the conv and the gated
  * delta rule advanced position by position -- and writes the logits of
@@ -183,7 +200,10 @@ int mk_verify(mk_engine *e, const int32_t *tokens_host, int n,
 
 /* Keep the first n_keep (1..n) positions of the last mk_verify: the state
  * becomes the checkpoint after position n_keep-1 and the position advances
- * by n_keep.  MK_ERR_STATE if no verify is pending. */
+ * by n_keep (the rollback of rejected draft tokens that exact greedy
+ * speculative decoding needs; same follow-up post, accuracy paragraph:
+ * greedy output stays the main model's greedy choice).
+ * MK_ERR_STATE if no verify is pending. */
 int mk_accept(mk_engine *e, int n_keep);
 
 /* Current position (number of tokens consumed). */
@@ -221,8 +241,9 @@ int64_t mk_launch_count(const mk_engine *e);
  * MK_ERR_TIMEOUT and the kernel returns early.  `fail_phase` >= 0 makes the
  * next decode launch wait, in that phase (0-based index of the launch's
  * phase sequence: five phases per layer, then the LM head), for data
- * tagged with a value no phase ever writes, so the wait
- * must run out (tests of the timeout path only). */
+ * tagged with a value no phase ever writes (or a split-K sum with one
+ * contribution more than any phase adds), so the wait must run out (tests
+ * of the timeout path only). */
 int mk_debug_set_wait_limit(mk_engine *e, int64_t limit_ns, int fail_phase);
 
 /* ------------------------------------------------------------------------
@@ -240,6 +261,27 @@ int mk_delta_step(float *S, const void *q, const void *k, const void *v,
                   const float *alpha, const float *beta, float *o, int B,
                   int heads, int dk, int dv, void *stream);
 
+/* The gated delta rule over a whole sequence of T positions in the
+ * chunkwise-parallel form the prompt path uses ("Gated Delta Networks",
+ * the WY / UT representation of a chunk of delta-rule updates: chunks of 64
+ * positions prepared independently, then one pass over the chunks per slice
+ * of state rows), no engine.  Results equal T consecutive steps of
+ * mk_delta_step up to rounding.
+ *   S      device float32 [heads][dv][dk], read and written
+ *   q, k   device float32 [heads][T][dk], used as given (no renormalisation)
+ *   v      device float32 [heads][T][dv]
+ *   alpha, beta device float32 [heads][T]
+ *   o      device float32 [heads][T][dv]   (o_t = S_t q_t)
+ *   workspace device scratch, 16-byte aligned, at least
+ *          mk_delta_chunked_ws_bytes(T, heads, dk) bytes (caller-owned)
+ * dk == dv in {64, 128} (else MK_ERR_UNSUPPORTED); MK_ERR_ARG on NULL,
+ * misaligned or short arguments.  Asynchronous on `stream`. */
+size_t mk_delta_chunked_ws_bytes(int T, int heads, int dk);
+int mk_delta_chunked(float *S, const float *q, const float *k, const float *v,
+                     const float *alpha, const float *beta, float *o, int T,
+                     int heads, int dk, int dv, void *workspace, size_t ws_bytes,
+                     void *stream);
+
 /* Debug: the prompt path's tensor-core GEMM on its own, asynchronous on
  * `stream` (a cudaStream_t, may be NULL):
  *   C[t][n] = sum_k (X_hi[t][k] + X_lo[t][k]) * W[n][k]
@@ -250,7 +292,10 @@ int mk_delta_step(float *S, const void *q, const void *k, const void *v,
  * MK_ERR_ARG on bad sizes, MK_ERR_UNSUPPORTED if the TMA descriptors cannot
  * be encoded.  The first call on a device allocates a 4-byte device word
  * (kept for the life of the process) where a device-side wait that runs
- * out is recorded; it is not reported. */
+ * out is recorded.  Every call clears that word first (stream-ordered), and
+ * if a tile's wait runs out, all of C is set to NaN: the call returns
+ * before the GPU runs it, so a timed-out call shows in its output, never as
+ * silently wrong values. */
 int mk_debug_gemm(const void *W, const void *X, float *C, int n_out, int T,
                   int K, void *stream);
 
@@ -264,10 +309,12 @@ int mk_debug_gemm(const void *W, const void *X, float *C, int n_out, int T,
  * rules and layouts as mk_debug_gemm.  The first call on a device (made
  * with that device current) looks up the scratch address with
  * cudaGetSymbolAddress; make that first call before any stream capture.
- * Nothing needs to start at zero: every partial is written before it is
- * read, and the private wait-error word starts at zero when the library
- * loads.  Calls share the scratch, so calls that overlap (other streams or
- * threads without ordering) race; serialise them. */
+ * No partial needs to start at zero: every partial is written before it is
+ * read.  The private wait-error word (also static) is cleared by every call
+ * with cudaMemsetAsync before its kernels; if a range's wait runs out it is
+ * set, and the reduction writes NaN to all of C instead of the sums.  Calls
+ * share the scratch, so calls that overlap (other streams or threads
+ * without ordering) race; serialise them. */
 int mk_debug_gemm_noalloc(const void *W, const void *X, float *C, int n_out,
                           int T, int K, void *stream);
 
