@@ -1293,7 +1293,7 @@ __device__ __forceinline__ bool att_merge_block(const DevModel& M, int S, int e0
 // Cursor over one CTA's chunk schedule for one launch: every phase of every
 // layer, then the LM head, each split into chunks of at most `rpc` rows.
 // ----------------------------------------------------------------------------
-constexpr size_t PF_AHEAD = size_t(64) << 10;  // L2 prefetch distance per CTA (bytes)
+constexpr size_t PF_AHEAD = size_t(128) << 10;  // L2 prefetch distance per CTA (bytes)
 
 struct ChunkCursor {
   const PD* tab;

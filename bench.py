@@ -30,9 +30,10 @@ GEN = 128
 # DRAM bytes (read + written) of one decode launch at context 520, from an ncu
 # capture of the current decode kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum); None once the kernel changes.
-DECODE_TRAFFIC_BYTES = 1.3223e9
+DECODE_TRAFFIC_BYTES = None
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 
 
 def parse_args():
@@ -44,26 +45,32 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extras", action="store_true",
                    help="skip the long-context, verify, prefill-roofline and delta-sweep lines")
-    p.add_argument("--mode", choices=["full", "kernel"], default="full",
-                   help="kernel: W+K single decode launches at context 520 on a "
-                        "seeded synthetic state (small case for profilers)")
+    p.add_argument("--mode", choices=["full", "kernel", "delta", "verify"], default="full",
+                   help="small cases for profilers: kernel = W+K single decode launches "
+                        "at context --ctx on a seeded synthetic state; delta = W+K "
+                        "isolated delta steps at batch --batch; verify = W+K 5-token "
+                        "verify calls at context 4096")
+    p.add_argument("--ctx", type=int, default=520, help="context of --mode kernel")
+    p.add_argument("--batch", type=int, default=8, help="sequences of --mode delta")
     return p.parse_args()
 
 
 def run_kernel_mode(args):
-    """W warm-up + K timed decode launches at context 520 (one engine)."""
+    """W warm-up + K timed decode launches at context --ctx (one engine)."""
     import numpy as np
     import torch
 
     import attention_decode_megakernel_b200 as mk
     from attention_decode_megakernel_b200 import build, synth
     build.build()
-    cfg = synth.hybrid_08b_config(max_ctx=PROMPT + 64)
+    ctx = args.ctx
+    cfg = synth.hybrid_08b_config(max_ctx=ctx + 64)
     w = synth.make_weights(cfg)
     eng = mk.Engine(cfg, w)
-    st = synth.make_engine_state(cfg, ctx=PROMPT)
+    st = synth.make_engine_state(cfg, ctx=ctx)
     dev = {k: (torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v).cuda()
                if isinstance(v, np.ndarray) else v) for k, v in st.items()}
+    del st
     eng.set_state(dev)
     logits = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
     for _ in range(args.warmup):
@@ -76,9 +83,79 @@ def run_kernel_mode(args):
     e1.record(eng.stream)
     eng.sync()
     ms = e0.elapsed_time(e1) / max(args.steps, 1)
-    print(json.dumps({"mode": "kernel", "launches": args.warmup + args.steps,
+    print(json.dumps({"mode": "kernel", "ctx": ctx, "launches": args.warmup + args.steps,
                       "ms_per_launch": ms,
-                      "GBps": decode_bytes(cfg, PROMPT + args.warmup) / ms / 1e6}), flush=True)
+                      "GBps": decode_bytes(cfg, ctx + args.warmup) / ms / 1e6}), flush=True)
+
+
+def run_delta_mode(args):
+    """W warm-up + K timed isolated delta steps, B = --batch sequences x 16
+    heads, dk = dv = 128 (one launch per step)."""
+    import torch
+
+    import attention_decode_megakernel_b200 as mk
+    from attention_decode_megakernel_b200 import build
+    build.build()
+    B, H, D = args.batch, 16, 128
+    S = torch.randn(B, H, D, D, device="cuda") * 0.1
+    q = torch.nn.functional.normalize(torch.randn(B, H, D, device="cuda"), dim=-1)
+    k = torch.nn.functional.normalize(torch.randn(B, H, D, device="cuda"), dim=-1)
+    q16, k16 = q.to(torch.bfloat16).view(torch.int16), k.to(torch.bfloat16).view(torch.int16)
+    v16 = torch.randn(B, H, D, device="cuda").to(torch.bfloat16).view(torch.int16)
+    be = torch.rand(B, H, device="cuda")
+    al = 0.9 + 0.1 * torch.rand(B, H, device="cuda")
+    o = torch.empty(B, H, D, device="cuda")
+    for _ in range(args.warmup):
+        mk.mk_delta_step(S, q16, k16, v16, al, be, o)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        mk.mk_delta_step(S, q16, k16, v16, al, be, o)
+    e1.record()
+    torch.cuda.synchronize()
+    us = 1000.0 * e0.elapsed_time(e1) / max(args.steps, 1)
+    sb = 2 * B * H * D * D * 4 + B * H * (3 * D * 2 + 8 + D * 4)
+    print(json.dumps({"mode": "delta", "batch": B, "us_per_step": us, "bytes_per_step": sb,
+                      "GBps": sb / us / 1e3}), flush=True)
+
+
+def run_verify_mode(args):
+    """W warm-up + K timed 5-token verify calls (accept 1 each) at context
+    4096 of the 0.8B-shaped model on a seeded synthetic state."""
+    import numpy as np
+    import torch
+
+    import attention_decode_megakernel_b200 as mk
+    from attention_decode_megakernel_b200 import build, synth
+    build.build()
+    ctx = 4096
+    cfg = synth.hybrid_08b_config(max_ctx=ctx + 64)
+    w = synth.make_weights(cfg)
+    eng = mk.Engine(cfg, w)
+    st = synth.make_engine_state(cfg, ctx=ctx)
+    eng.set_state({k: (torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v).cuda()
+                       if isinstance(v, np.ndarray) else v) for k, v in st.items()})
+    del st
+    drafts = synth.make_tokens(cfg.vocab, 5 * (args.warmup + args.steps),
+                               seed=synth.SEED_DRAFTS).reshape(-1, 5)
+    vl = torch.empty((5, cfg.vocab), dtype=torch.float32, device="cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = 0
+    for i in range(args.warmup + args.steps):
+        if i == args.warmup:
+            eng.sync()
+            n0 = eng.launch_count()
+            e0.record(eng.stream)
+        eng.verify(drafts[i], vl)
+        eng.accept(1)
+    e1.record(eng.stream)
+    eng.sync()
+    ms = e0.elapsed_time(e1) / max(args.steps, 1)
+    print(json.dumps({"mode": "verify", "ctx": ctx, "calls": args.warmup + args.steps,
+                      "ms_per_call": ms,
+                      "launches_per_call": (eng.launch_count() - n0) / max(args.steps, 1)}),
+          flush=True)
 
 
 def peaks():
@@ -89,6 +166,18 @@ def peaks():
         return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def sustained_tc_peak():
+    """bf16 tensor throughput sustained under the power cap (the prompt path
+    runs inside a seconds-long loop), else the burst figure."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops_sustained"]), "measured sustained"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback sustained"
 
 
 def decode_bytes(cfg, ctx):
@@ -324,11 +413,12 @@ def extra_workloads(mk, synth, torch, np, prefill_ms_per_call, hbm, tc_peak, pea
     cfg = synth.hybrid_08b_config(max_ctx=PROMPT + GEN + 8)
     flops = 2.0 * matrix_params(cfg) * PROMPT + 2.0 * cfg.vocab * cfg.hidden
     tf = flops / (prefill_ms_per_call / 1000.0) / 1e12
+    tc_sus, sus_kind = sustained_tc_peak()
     out["prefill_pp520"] = {"tok_s": PROMPT / (prefill_ms_per_call / 1000.0),
                             "ms": prefill_ms_per_call, "gflop": flops / 1e9,
-                            "roofline": {"bound": "tensor", "achieved": tf, "peak": tc_peak,
-                                         "unit": "TFLOP/s", "frac": tf / tc_peak,
-                                         "peak_kind": peak_kind}}
+                            "roofline": {"bound": "tensor", "achieved": tf, "peak": tc_sus,
+                                         "unit": "TFLOP/s", "frac": tf / tc_sus,
+                                         "peak_kind": sus_kind, "burst_peak": tc_peak}}
     del cfg
 
     # long context: the attention layers' KV at 32768 positions (synthetic
@@ -403,7 +493,8 @@ def extra_workloads(mk, synth, torch, np, prefill_ms_per_call, hbm, tc_peak, pea
     del eng, w
 
     # isolated gated delta-rule step: B sequences x 16 heads, dk = dv = 128,
-    # 1024 sequential steps, one launch per step
+    # 1024 sequential steps, one launch per step, the 1024 launches replayed
+    # from one CUDA graph (the device time, not the host's launch rate)
     sweep = {}
     for B in (1, 8, 64):
         H, D, steps = 16, 128, 1024
@@ -418,15 +509,24 @@ def extra_workloads(mk, synth, torch, np, prefill_ms_per_call, hbm, tc_peak, pea
         for t in range(16):
             mk.mk_delta_step(S, q16[t % 8], k16[t % 8], v16[t % 8], al[t % 8], be[t % 8], o)
         torch.cuda.synchronize()
+        cs = torch.cuda.Stream()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cs):
+            for t in range(steps):
+                mk.mk_delta_step(S, q16[t % 8], k16[t % 8], v16[t % 8], al[t % 8], be[t % 8], o,
+                                 stream=cs.cuda_stream)
+        graph.replay()  # warm-up replay (replays run on the current stream)
+        torch.cuda.synchronize()
         e0.record()
-        for t in range(steps):
-            mk.mk_delta_step(S, q16[t % 8], k16[t % 8], v16[t % 8], al[t % 8], be[t % 8], o)
+        graph.replay()
         e1.record()
         torch.cuda.synchronize()
         us = 1000.0 * e0.elapsed_time(e1) / steps
+        del graph
         sb = 2 * B * H * D * D * 4 + B * H * (3 * D * 2 + 8 + D * 4)
         sweep["B%d" % B] = {"us_per_step": us, "state_GBps": sb / us / 1e3,
-                            "frac": sb / us / 1e3 / hbm, "bytes_per_step": sb}
+                            "frac": sb / us / 1e3 / hbm, "bytes_per_step": sb,
+                            "launch": "CUDA graph of %d launches" % steps}
         del S, q, k, q16, k16, v16, be, al, o
     out["delta_sweep_dk128_h16"] = sweep
     return out
@@ -439,6 +539,12 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.mode == "delta":
+        run_delta_mode(args)
+        return
+    if args.mode == "verify":
+        run_verify_mode(args)
         return
     if args.mode == "kernel":
         run_kernel_mode(args)
