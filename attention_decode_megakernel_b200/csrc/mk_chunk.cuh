@@ -232,6 +232,7 @@ template <int DK>
 __global__ void __launch_bounds__(SCAN_THREADS, 1) chunk_scan_kernel(
     float* __restrict__ S, const float* __restrict__ prep, int T, float* __restrict__ O,
     size_t o_ts, size_t o_hs) {
+  griddep_launch_dependents();
   extern __shared__ __align__(16) float sm[];
   constexpr int R = SCAN_ROWS, LD = DK + 4, LC = C + 4;
   using B = Blk<DK>;

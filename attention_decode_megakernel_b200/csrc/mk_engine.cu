@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstring>
 #include <new>
+#include <utility>
 
 #include "mk.h"
 #include "mk_chunk.cuh"
@@ -13,6 +14,8 @@
 #include "mk_delta.cuh"
 #include "mk_model.cuh"
 #include "mk_prefill.cuh"
+#include "mk_skinny.cuh"
+#include "mk_verify.cuh"
 
 namespace {
 
@@ -34,6 +37,9 @@ struct Layout {
   int tmax, pw, aw;
   size_t pf_tok, pf_x, pf_xn, pf_p, pf_c, pf_o, pf_a16, pf_qk, pf_bak, pf_att, pf_part;
   size_t pf_chunk;  // chunkwise delta rule operands: [nh][chunks][block]
+  // verify records, two sets: keys, values [n_dn][kMaxVerify][nh][dk],
+  // {alpha, beta} [n_dn][kMaxVerify][nh], conv inputs [n_dn][kMaxVerify][ch]
+  size_t vlog_k[2], vlog_v[2], vlog_ab[2], vlog_u[2];
   size_t total;
 };
 
@@ -121,13 +127,23 @@ Layout make_layout(const mk_config& c) {
     L.pf_qk = take(size_t(c.dn_heads) * T * 2 * c.dn_dk * 4);
     L.pf_bak = take(size_t(c.dn_heads) * T * 16);
     // key-split attention partials of a short chunk: [t][q head][range][hd + 2]
-    const size_t nsplit = (size_t(c.max_ctx) + mk::pf::ATT_SPLIT_LEN - 1) / mk::pf::ATT_SPLIT_LEN;
+    const size_t rlen = mk::pf::ATT_SPLIT_LEN < mk::vf::ATT_L ? mk::pf::ATT_SPLIT_LEN : mk::vf::ATT_L;
+    const size_t nsplit = (size_t(c.max_ctx) + rlen - 1) / rlen;
     L.pf_att = take(size_t(mk::kMaxVerify) * c.q_heads * nsplit * (c.head_dim + 2) * 4);
     // split-K partial sums of a prompt GEMM with few output tiles (< 100):
     // k_split x T x n_out <= (148 + tiles) x 128 x 128 floats
     L.pf_part = take(size_t(kSplitPartialTiles) * mk::pf::BM * mk::pf::BN * 4);
     const size_t blk = c.dn_dk == 64 ? mk::ck::Blk<64>::FLOATS : mk::ck::Blk<128>::FLOATS;
     L.pf_chunk = take(size_t(c.dn_heads) * ((T + mk::ck::C - 1) / mk::ck::C) * blk * 4);
+  }
+  {
+    const size_t n_dn = size_t(c.n_layers - count_attn(c)), V = mk::kMaxVerify;
+    for (int sel = 0; sel < 2; ++sel) {
+      L.vlog_k[sel] = take(n_dn * V * c.dn_heads * c.dn_dk * 4);
+      L.vlog_v[sel] = take(n_dn * V * c.dn_heads * c.dn_dv * 4);
+      L.vlog_ab[sel] = take(n_dn * V * c.dn_heads * 8);
+      L.vlog_u[sel] = take(n_dn * V * ch * 4);
+    }
   }
   L.total = off;
   return L;
@@ -213,11 +229,17 @@ struct mk_engine {
   bool amax_valid;  // the last launch was a decode step at the current position
   int pending_verify;
   int verify_bufs[mk::kMaxVerify];
+  // verify by records (the chunk path): the pending verify wrote record set
+  // vlog_sel; after mk_accept the first replay_n records of set replay_sel
+  // are applied to the state by the next call that reads it
+  bool verify_logged;
+  int vlog_sel, replay_n, replay_sel;
   int64_t launches;
   long long wait_ns;
   int fail_phase;
   // multi-token prompt path
   bool pf_ok;
+  bool sk_ok;  // the skinny projections fit (verify chunks and prompts of <= 8 tokens)
   struct LayerMaps {
     CUtensorMap in_proj, out, q, k, v, gate, up, down;
   } maps[MK_MAX_LAYERS];
@@ -281,7 +303,11 @@ int launch_decode(mk_engine* e, int pos, int st_in, int st_out, int token, int t
 
 // One decode launch at the current position that advances the state: it
 // reads the current state buffer and writes the next one in the ring.
+int replay_pending(mk_engine* e);
+
 int decode_advance(mk_engine* e, int token, int tok_src, float* logits, int32_t* tok_out) {
+  const int rp = replay_pending(e);
+  if (rp != MK_OK) return rp;
   const int nxt = (e->cur_buf + 1) % mk::kStateBufs;
   const int rc = launch_decode(e, e->pos, e->cur_buf, nxt, token, tok_src, logits, tok_out);
   if (rc == MK_OK) {
@@ -351,12 +377,130 @@ int launch_gemm(mk_engine* e, const CUtensorMap& tw, const CUtensorMap& tx, floa
   return cuda_status(cudaGetLastError());
 }
 
+// A launch that may start while the kernel before it in the stream is
+// still running (programmatic stream serialisation); the kernel calls
+// griddep_wait() before it reads what that kernel writes.
+template <typename... KArgs, typename... Act>
+int launch_pdl(mk_engine* e, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+               Act&&... args) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = grid;
+  lc.blockDim = block;
+  lc.dynamicSmemBytes = smem;
+  lc.stream = e->stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  const cudaError_t r = cudaLaunchKernelEx(&lc, kern, std::forward<Act>(args)...);
+  e->launches += 1;
+  return cuda_status(r);
+}
+
+// One skinny projection (a chunk of T <= 8 tokens): grid of at most two
+// CTAs per SM over the output's row blocks, launched so that it may start
+// (and stream its first weights) while the kernel before it finishes.
+int launch_skinny(mk_engine* e, mk::sk::Args a) {
+  a.kw = mk::sk::pick_kw(a.K);
+  a.err = e->hm.err;
+  a.wait_ns = e->wait_ns;
+  const int rpb = (mk::sk::WARPS / a.kw) * mk::sk::RW;
+  const int lpb = a.pair ? rpb / 2 : rpb;
+  const int nblk = (a.N + lpb - 1) / lpb;
+  return launch_pdl(e, mk::sk::skinny_gemv_kernel, dim3(nblk < mk::sk::MAX_CTAS ? nblk : mk::sk::MAX_CTAS),
+                    dim3(mk::sk::THREADS), mk::sk::smem_bytes(a.mode, a.T, a.K, a.dv), a);
+}
+
+// Record set `sel` of DeltaNet layer `sub`.
+mk::vf::Log vlog(mk_engine* e, int sel, int sub) {
+  const Layout& L = e->lay;
+  const mk::DevModel& m = e->hm;
+  const size_t V = mk::kMaxVerify;
+  mk::vf::Log g;
+  g.k = reinterpret_cast<float*>(e->ws + L.vlog_k[sel]) + size_t(sub) * V * m.nh * m.dk;
+  g.v = reinterpret_cast<float*>(e->ws + L.vlog_v[sel]) + size_t(sub) * V * m.nh * m.dv;
+  g.ab = reinterpret_cast<float2*>(e->ws + L.vlog_ab[sel]) + size_t(sub) * V * m.nh;
+  g.u = reinterpret_cast<float*>(e->ws + L.vlog_u[sel]) + size_t(sub) * V * m.ch;
+  return g;
+}
+
+// What a verify chunk replays first (R records of set rsel, the replayed
+// state going to buffer nb) and where it writes its own records (set wsel).
+struct VerifyPlan {
+  int R, rsel, wsel, nb;
+};
+
+// Arguments of dn_verify_kernel for DeltaNet layer `sub` (layer 0 plus the
+// per-layer strides for a launch over all layers): the state and conv
+// history of the current buffer, replayed into buffer nb.
+mk::vf::DnArgs dn_args(mk_engine* e, int sub, int R, int rsel, int nb) {
+  const mk::DevModel& m = e->hm;
+  const size_t soff = size_t(sub) * m.nh * m.dv * m.dk, coff = size_t(sub) * m.ch;
+  const size_t V = mk::kMaxVerify;
+  mk::vf::DnArgs a{};
+  a.S_in = m.dn_state[e->cur_buf] + soff;
+  a.S_out = m.dn_state[nb] + soff;
+  a.conv_in = reinterpret_cast<const float4*>(m.conv_state[e->cur_buf]) + coff;
+  a.conv_out = reinterpret_cast<float4*>(m.conv_state[nb]) + coff;
+  a.rlog = vlog(e, rsel, sub);
+  a.R = R;
+  a.s_stride = size_t(m.nh) * m.dv * m.dk;
+  a.c_stride = size_t(m.ch);
+  a.lk_stride = V * m.nh * m.dk;
+  a.lab_stride = V * m.nh;
+  a.lu_stride = V * m.ch;
+  a.nh = m.nh;
+  a.ch = m.ch;
+  return a;
+}
+
+// A verify chunk (a.T > 0) may start while the kernel before it finishes and
+// runs the CTAs of each head as one cluster when it applies the gated norm;
+// a replay (a.T == 0) is a plain launch over all layers.
+int launch_dn_verify(mk_engine* e, const mk::vf::DnArgs& a, dim3 grid) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = grid;
+  lc.blockDim = dim3(mk::vf::THREADS);
+  lc.stream = e->stream;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;
+  at[1].val.clusterDim.x = 1;
+  at[1].val.clusterDim.y = grid.y;
+  at[1].val.clusterDim.z = 1;
+  lc.attrs = at;
+  lc.numAttrs = a.T == 0 ? 0 : a.out_norm ? 2 : 1;
+  const cudaError_t r = e->hm.dk == 128 ? cudaLaunchKernelEx(&lc, mk::vf::dn_verify_kernel<128>, a)
+                                        : cudaLaunchKernelEx(&lc, mk::vf::dn_verify_kernel<64>, a);
+  e->launches += 1;
+  return cuda_status(r);
+}
+
+// Apply the accepted records of the last verify to the state (into the next
+// state buffer) before a call that reads the state in another way.
+int replay_pending(mk_engine* e) {
+  if (e->replay_n == 0) return MK_OK;
+  const mk::DevModel& m = e->hm;
+  const int nb = (e->cur_buf + 1) % mk::kStateBufs;
+  if (m.n_dn > 0) {
+    const mk::vf::DnArgs a = dn_args(e, 0, e->replay_n, e->replay_sel, nb);
+    const int rc = launch_dn_verify(e, a, dim3(m.nh, m.dv / mk::vf::BR, m.n_dn));
+    if (rc != MK_OK) return rc;
+  }
+  e->cur_buf = nb;
+  e->replay_n = 0;
+  return MK_OK;
+}
+
 // The stack over T positions starting at e->pos through the chunk kernels.
-// Prompt chunk (ck_bufs == nullptr): the state is updated in place and the
-// position advances.  Verify chunk: the state after position t goes to state
-// buffer ck_bufs[t], the current state is left as it was, the position does
-// not move, and logits_out [T][vocab] receives every position's logits.
-int run_chunk(mk_engine* e, const int32_t* tokens_host, int T, const int* ck_bufs,
+// Prompt chunk (vp == nullptr): the state is updated in place and the
+// position advances.  Verify chunk: the pending records are replayed into
+// buffer vp->nb (when vp->R > 0), the chunk writes its records to set
+// vp->wsel and no state, the position does not move, and logits_out
+// [T][vocab] receives every position's logits.
+int run_chunk(mk_engine* e, const int32_t* tokens_host, int T, const VerifyPlan* vp,
               float* logits_out) {
   using namespace mk::pf;
   const mk_config& c = e->cfg;
@@ -376,6 +520,34 @@ int run_chunk(mk_engine* e, const int32_t* tokens_host, int T, const int* ck_buf
   uint16_t* A16 = reinterpret_cast<uint16_t*>(ws + L.pf_a16);
   float* QK = reinterpret_cast<float*>(ws + L.pf_qk);
   float4* BAK = reinterpret_cast<float4*>(ws + L.pf_bak);
+  // at most 8 tokens: every projection is one weight-streaming pass with its
+  // operand's producer (RMSNorm, SwiGLU, gated norm) fused into its prologue
+  const bool sk = T <= mk::sk::TMAX && e->sk_ok;
+  // fp32 view of the bf16 operand buffer: the attention output and SiLU(gate)
+  // * up of a skinny chunk, [T][aw]
+  float* Af = reinterpret_cast<float*>(A16);
+  auto sk_norm = [&](const uint16_t* W0, const uint16_t* W1, int N, const uint16_t* gain,
+                     float* C, int ldc) {
+    mk::sk::Args a{};
+    a.W0 = W0;
+    a.W1 = W1;
+    a.pair = W1 != nullptr;
+    a.N = N;
+    a.K = H;
+    a.T = T;
+    a.mode = mk::sk::X_NORM;
+    a.X = X;
+    a.ldx = H;
+    a.gain = gain;
+    a.eps = c.rms_eps;
+    a.C = C;
+    a.ldc = ldc;
+    return launch_skinny(e, a);
+  };
+  if (!vp) {
+    const int rp = replay_pending(e);
+    if (rp != MK_OK) return rp;
+  }
   cudaError_t r = cudaMemcpyAsync(tok, tokens_host, size_t(T) * 4, cudaMemcpyHostToDevice, st);
   if (r != cudaSuccess) return cuda_status(r);
   embed_kernel<<<T, ROW_THREADS, 0, st>>>(tok, m.embed, X, H);
@@ -384,31 +556,39 @@ int run_chunk(mk_engine* e, const int32_t* tokens_host, int T, const int* ck_buf
   for (int l = 0; l < c.n_layers && rc == MK_OK; ++l) {
     const mk::DevLayer& D = m.layers[l];
     const mk_engine::LayerMaps& mp = e->maps[l];
-    rmsnorm_bf16_kernel<<<T, ROW_THREADS, 0, st>>>(X, D.attn_norm, Xn, H, c.rms_eps, lo_x);
+    if (!sk) rmsnorm_bf16_kernel<<<T, ROW_THREADS, 0, st>>>(X, D.attn_norm, Xn, H, c.rms_eps, lo_x);
     if (!D.is_attn) {
-      rc = launch_gemm(e, mp.in_proj, e->map_xn, P, pw, m.rin, T, H, 0);
-      mk::pf::Ckpt ckc{}, cks{};
-      if (ck_bufs)
-        for (int t = 0; t < T; ++t) {
-          ckc.p[t] = m.conv_state[ck_bufs[t]] + size_t(D.sub) * m.ch * 4;
-          cks.p[t] = m.dn_state[ck_bufs[t]] + size_t(D.sub) * nh * dv * dk;
-        }
-      float4* cst = reinterpret_cast<float4*>(m.conv_state[e->cur_buf]) + size_t(D.sub) * m.ch;
-      float* Cv = reinterpret_cast<float*>(ws + L.pf_c);
-      conv_kernel<<<dim3((m.ch + 255) / 256, T), 256, 0, st>>>(P, pw, cst, D.conv_w, m.ch, Cv,
-                                                              m.ch, ckc);
-      if (!ck_bufs) {
+      rc = sk ? sk_norm(D.in_proj, nullptr, m.rin, D.attn_norm, P, pw)
+              : launch_gemm(e, mp.in_proj, e->map_xn, P, pw, m.rin, T, H, 0);
+      if (vp) {
+        // verify: replay, conv, gates and recurrence in one kernel, which
+        // records the chunk's positions instead of writing states
+        mk::vf::DnArgs a = dn_args(e, D.sub, vp->R, vp->rsel, vp->nb);
+        a.wlog = vlog(e, vp->wsel, D.sub);
+        a.P = P;
+        a.ldp = pw;
+        a.conv_w = D.conv_w;
+        a.A_log = D.A_log;
+        a.dt_bias = D.dt_bias;
+        a.O = O;
+        a.ldo = nh * dv;
+        a.out_norm = sk ? D.out_norm : nullptr;  // else the gated norm kernel below
+        a.eps = c.rms_eps;
+        a.zcol = m.ch;
+        a.T = T;
+        if (rc == MK_OK) rc = launch_dn_verify(e, a, dim3(nh, dv / mk::vf::BR));
+      } else {
+        float4* cst = reinterpret_cast<float4*>(m.conv_state[e->cur_buf]) + size_t(D.sub) * m.ch;
+        float* Cv = reinterpret_cast<float*>(ws + L.pf_c);
+        conv_kernel<<<dim3((m.ch + 255) / 256, T), 256, 0, st>>>(P, pw, cst, D.conv_w, m.ch, Cv,
+                                                                m.ch);
         conv_state_kernel<<<(m.ch + 255) / 256, 256, 0, st>>>(P, pw, cst, m.ch, T);
-        e->launches += 1;
-      }
-      dn_prep_kernel<<<dim3(T, nh), dk, 0, st>>>(Cv, m.ch, P, pw, nh, dk, m.ch, dv, D.A_log,
-                                                 D.dt_bias, QK, BAK, T);
-      float* S = m.dn_state[e->cur_buf] + size_t(D.sub) * nh * dv * dk;
-      const dim3 rgrid(nh, dv / (REC_WARPS * REC_RPW));
-      const int vcol = 2 * nh * dk;
-      if (!ck_bufs) {
-        // prompt chunk: the chunkwise-parallel form (independent per
-        // chunk of 64 positions, then one pass over the chunks)
+        dn_prep_kernel<<<dim3(T, nh), dk, 0, st>>>(Cv, m.ch, P, pw, nh, dk, m.ch, dv, D.A_log,
+                                                   D.dt_bias, QK, BAK, T);
+        float* S = m.dn_state[e->cur_buf] + size_t(D.sub) * nh * dv * dk;
+        const int vcol = 2 * nh * dk;
+        // the chunkwise-parallel form (independent per chunk of 64
+        // positions, then one pass over the chunks)
         float* prep = reinterpret_cast<float*>(ws + L.pf_chunk);
         const dim3 pg((T + mk::ck::C - 1) / mk::ck::C, nh), sg(dv / mk::ck::SCAN_ROWS, nh);
         if (dk == 128) {
@@ -422,26 +602,83 @@ int run_chunk(mk_engine* e, const int32_t* tokens_host, int T, const int* ck_buf
           mk::ck::chunk_scan_kernel<64><<<sg, mk::ck::SCAN_THREADS, mk::ck::scan_smem<64>(), st>>>(
               S, prep, T, O, size_t(nh) * dv, size_t(dv));
         }
-        e->launches += 1;  // two kernels where the scan was one
-      } else if (dk == 128 && ck_bufs)
-        recurrence_kernel<128, true><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, Cv, m.ch, vcol,
-                                                                       O, nh * dv, T, cks);
-      else
-        recurrence_kernel<64, true><<<rgrid, REC_WARPS * 32, 0, st>>>(S, QK, BAK, Cv, m.ch, vcol,
-                                                                      O, nh * dv, T, cks);
-      gated_norm_kernel<<<dim3(T, nh), dv, 0, st>>>(O, nh * dv, P, pw, m.ch, D.out_norm, A16, aw,
-                                                    c.rms_eps, lo_a);
-      if (rc == MK_OK) rc = launch_gemm(e, mp.out, e->map_a16_dn, X, H, H, T, nh * dv, 1);
+        e->launches += 5;  // conv, its state, gates, chunk prep and scan
+      }
+      if (sk) {
+        mk::sk::Args a{};
+        a.W0 = D.out_proj;
+        a.N = H;
+        a.K = nh * dv;
+        a.T = T;
+        // verify: O holds the gated-normed readout already
+        a.mode = vp ? mk::sk::X_COPY : mk::sk::X_GATED;
+        a.X = O;
+        a.ldx = nh * dv;
+        a.X2 = P + m.ch;  // z
+        a.ldx2 = pw;
+        a.dv = dv;
+        a.gain = D.out_norm;
+        a.eps = c.rms_eps;
+        a.C = X;
+        a.ldc = H;
+        a.accumulate = 1;
+        if (rc == MK_OK) rc = launch_skinny(e, a);
+      } else {
+        gated_norm_kernel<<<dim3(T, nh), dv, 0, st>>>(O, nh * dv, P, pw, m.ch, D.out_norm, A16,
+                                                      aw, c.rms_eps, lo_a);
+        if (rc == MK_OK) rc = launch_gemm(e, mp.out, e->map_a16_dn, X, H, H, T, nh * dv, 1);
+      }
     } else {
-      rc = launch_gemm(e, mp.q, e->map_xn, P, pw, nq * hd, T, H, 0);
-      if (rc == MK_OK) rc = launch_gemm(e, mp.k, e->map_xn, P + nq * hd, pw, nkv * hd, T, H, 0);
-      if (rc == MK_OK)
-        rc = launch_gemm(e, mp.v, e->map_xn, P + (nq + nkv) * hd, pw, nkv * hd, T, H, 0);
+      if (sk) {
+        rc = sk_norm(D.w_qkv, nullptr, (nq + 2 * nkv) * hd, D.attn_norm, P, pw);
+      } else {
+        rc = launch_gemm(e, mp.q, e->map_xn, P, pw, nq * hd, T, H, 0);
+        if (rc == MK_OK) rc = launch_gemm(e, mp.k, e->map_xn, P + nq * hd, pw, nkv * hd, T, H, 0);
+        if (rc == MK_OK)
+          rc = launch_gemm(e, mp.v, e->map_xn, P + (nq + nkv) * hd, pw, nkv * hd, T, H, 0);
+      }
       const size_t kvo = size_t(D.sub) * nkv * c.max_ctx * hd;
-      rope_kv_kernel<<<dim3(T, nq + nkv), hd / 2, 0, st>>>(P, pw, nq, nkv, hd, m.kc + kvo,
-                                                           m.vc + kvo, c.max_ctx, pos0,
-                                                           c.rope_theta);
-      if (T <= mk::kMaxVerify) {
+      if (sk && (nq / nkv) * T <= mk::vf::ATT_QMAX) {
+        // rope + KV append, the chunk attention over key ranges and their
+        // merge, each starting while the kernel before it finishes
+        if (rc == MK_OK)
+          rc = launch_pdl(e, rope_kv_kernel, dim3(T, nq + nkv), dim3(hd / 2), 0, P, pw, nq, nkv,
+                          hd, m.kc + kvo, m.vc + kvo, c.max_ctx, pos0, c.rope_theta);
+        mk::vf::AttArgs aa{};
+        aa.P = P;
+        aa.ldp = pw;
+        aa.kc = m.kc + kvo;
+        aa.vc = m.vc + kvo;
+        aa.max_ctx = c.max_ctx;
+        aa.nq = nq;
+        aa.nkv = nkv;
+        aa.pos0 = pos0;
+        aa.T = T;
+        aa.nsplit = (pos0 + T + mk::vf::ATT_L - 1) / mk::vf::ATT_L;
+        aa.part = reinterpret_cast<float*>(ws + L.pf_att);
+        aa.out = Af;
+        aa.ldo = aw;
+        const dim3 ag(aa.nsplit, nkv), mg(nq, T), tb(mk::vf::ATT_THREADS);
+        if (rc == MK_OK) {
+          if (hd == 256)
+            rc = launch_pdl(e, mk::vf::attn_chunk_kernel<256>, ag, tb, mk::vf::att_smem<256>(), aa);
+          else if (hd == 128)
+            rc = launch_pdl(e, mk::vf::attn_chunk_kernel<128>, ag, tb, mk::vf::att_smem<128>(), aa);
+          else
+            rc = launch_pdl(e, mk::vf::attn_chunk_kernel<64>, ag, tb, mk::vf::att_smem<64>(), aa);
+        }
+        if (rc == MK_OK) {
+          if (hd == 256)
+            rc = launch_pdl(e, mk::vf::attn_chunk_merge<256>, mg, tb, 0, aa);
+          else if (hd == 128)
+            rc = launch_pdl(e, mk::vf::attn_chunk_merge<128>, mg, tb, 0, aa);
+          else
+            rc = launch_pdl(e, mk::vf::attn_chunk_merge<64>, mg, tb, 0, aa);
+        }
+      } else if (T <= mk::kMaxVerify) {
+        rope_kv_kernel<<<dim3(T, nq + nkv), hd / 2, 0, st>>>(P, pw, nq, nkv, hd, m.kc + kvo,
+                                                             m.vc + kvo, c.max_ctx, pos0,
+                                                             c.rope_theta);
         // few queries: split the keys too, then merge the ranges
         float* part = reinterpret_cast<float*>(ws + L.pf_att);
         const int nsplit = (pos0 + T + ATT_SPLIT_LEN - 1) / ATT_SPLIT_LEN;
@@ -450,18 +687,25 @@ int run_chunk(mk_engine* e, const int32_t* tokens_host, int T, const int* ck_buf
         if (hd == 256) {
           attn_split_kernel<256><<<sg, ATT_SPLIT_WARPS * 32, 0, st>>>(
               P, pw, m.kc + kvo, m.vc + kvo, c.max_ctx, nq, nkv, pos0, nsplit, part);
-          attn_merge_kernel<256><<<mg, 256, 0, st>>>(part, nq, nsplit, A16, aw, lo_a);
+          attn_merge_kernel<256><<<mg, 256, 0, st>>>(part, nq, nsplit, A16, aw, lo_a,
+                                                      sk ? Af : nullptr);
         } else if (hd == 128) {
           attn_split_kernel<128><<<sg, ATT_SPLIT_WARPS * 32, 0, st>>>(
               P, pw, m.kc + kvo, m.vc + kvo, c.max_ctx, nq, nkv, pos0, nsplit, part);
-          attn_merge_kernel<128><<<mg, 128, 0, st>>>(part, nq, nsplit, A16, aw, lo_a);
+          attn_merge_kernel<128><<<mg, 128, 0, st>>>(part, nq, nsplit, A16, aw, lo_a,
+                                                      sk ? Af : nullptr);
         } else {
           attn_split_kernel<64><<<sg, ATT_SPLIT_WARPS * 32, 0, st>>>(
               P, pw, m.kc + kvo, m.vc + kvo, c.max_ctx, nq, nkv, pos0, nsplit, part);
-          attn_merge_kernel<64><<<mg, 64, 0, st>>>(part, nq, nsplit, A16, aw, lo_a);
+          attn_merge_kernel<64><<<mg, 64, 0, st>>>(part, nq, nsplit, A16, aw, lo_a,
+                                                      sk ? Af : nullptr);
         }
-        e->launches += 1;  // the merge
+        e->launches += 3;  // rope, key ranges, merge
       } else {
+        rope_kv_kernel<<<dim3(T, nq + nkv), hd / 2, 0, st>>>(P, pw, nq, nkv, hd, m.kc + kvo,
+                                                             m.vc + kvo, c.max_ctx, pos0,
+                                                             c.rope_theta);
+        e->launches += 2;  // rope, attention
         const dim3 agrid((T + 7) / 8, nq);
         if (hd == 256)
           attn_prefill_kernel<256><<<agrid, 256, 0, st>>>(P, pw, m.kc + kvo, m.vc + kvo,
@@ -476,26 +720,62 @@ int run_chunk(mk_engine* e, const int32_t* tokens_host, int T, const int* ck_buf
                                                          c.max_ctx, nq, nkv, pos0, T, A16, aw,
                                                          lo_a);
       }
-      if (rc == MK_OK) rc = launch_gemm(e, mp.out, e->map_a16_att, X, H, H, T, nq * hd, 1);
+      if (sk) {
+        mk::sk::Args a{};
+        a.W0 = D.w_o;
+        a.N = H;
+        a.K = nq * hd;
+        a.T = T;
+        a.mode = mk::sk::X_COPY;
+        a.X = Af;
+        a.ldx = aw;
+        a.C = X;
+        a.ldc = H;
+        a.accumulate = 1;
+        if (rc == MK_OK) rc = launch_skinny(e, a);
+      } else if (rc == MK_OK) {
+        rc = launch_gemm(e, mp.out, e->map_a16_att, X, H, H, T, nq * hd, 1);
+      }
     }
-    rmsnorm_bf16_kernel<<<T, ROW_THREADS, 0, st>>>(X, D.mlp_norm, Xn, H, c.rms_eps, lo_x);
-    if (rc == MK_OK) rc = launch_gemm(e, mp.gate, e->map_xn, P, pw, I, T, H, 0);
-    if (rc == MK_OK) rc = launch_gemm(e, mp.up, e->map_xn, P + I, pw, I, T, H, 0);
-    swiglu_kernel<<<dim3((I + 255) / 256, T), 256, 0, st>>>(P, pw, I, A16, aw, lo_a);
-    if (rc == MK_OK) rc = launch_gemm(e, mp.down, e->map_a16_mlp, X, H, H, T, I, 1);
-    e->launches += D.is_attn ? 5 : 7;  // besides the GEMMs
+    if (sk) {
+      if (rc == MK_OK) rc = sk_norm(D.w_gate, D.w_up, I, D.mlp_norm, Af, aw);
+      mk::sk::Args a{};
+      a.W0 = D.w_down;
+      a.N = H;
+      a.K = I;
+      a.T = T;
+      a.mode = mk::sk::X_COPY;
+      a.X = Af;
+      a.ldx = aw;
+      a.C = X;
+      a.ldc = H;
+      a.accumulate = 1;
+      if (rc == MK_OK) rc = launch_skinny(e, a);
+
+    } else {
+      rmsnorm_bf16_kernel<<<T, ROW_THREADS, 0, st>>>(X, D.mlp_norm, Xn, H, c.rms_eps, lo_x);
+      if (rc == MK_OK) rc = launch_gemm(e, mp.gate, e->map_xn, P, pw, I, T, H, 0);
+      if (rc == MK_OK) rc = launch_gemm(e, mp.up, e->map_xn, P + I, pw, I, T, H, 0);
+      swiglu_kernel<<<dim3((I + 255) / 256, T), 256, 0, st>>>(P, pw, I, A16, aw, lo_a);
+      if (rc == MK_OK) rc = launch_gemm(e, mp.down, e->map_a16_mlp, X, H, H, T, I, 1);
+      e->launches += D.is_attn ? 3 : 4;  // norms, SwiGLU (and the gated norm)
+    }
   }
   if (rc != MK_OK) return rc;
   if (logits_out) {
     // final norm and the tied LM head for every position of the chunk
-    rmsnorm_bf16_kernel<<<T, ROW_THREADS, 0, st>>>(X, m.final_norm, Xn, H, c.rms_eps, lo_x);
-    e->launches += 1;
-    rc = launch_gemm(e, e->map_embed, e->map_xn, logits_out, c.vocab, c.vocab, T, H, 0);
+    if (sk) {
+      rc = sk_norm(m.embed, nullptr, c.vocab, m.final_norm, logits_out, c.vocab);
+    } else {
+      rmsnorm_bf16_kernel<<<T, ROW_THREADS, 0, st>>>(X, m.final_norm, Xn, H, c.rms_eps, lo_x);
+      e->launches += 1;
+      rc = launch_gemm(e, e->map_embed, e->map_xn, logits_out, c.vocab, c.vocab, T, H, 0);
+    }
     if (rc != MK_OK) return rc;
   }
   r = cudaGetLastError();
   if (r != cudaSuccess) return cuda_status(r);
-  if (!ck_bufs) e->pos += T;
+  if (!vp) e->pos += T;
   return MK_OK;
 }
 
@@ -768,6 +1048,36 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
              cudaFuncSetAttribute(mk::pf::gemm_tc_partial,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   int(mk::pf::GEMM_SMEM)) == cudaSuccess;
+  {
+    // widest K of a skinny projection: hidden, MLP, DeltaNet readout, attention
+    int kmax = c.hidden;
+    if (c.mlp > kmax) kmax = c.mlp;
+    if (c.dn_heads * c.dn_dv > kmax) kmax = c.dn_heads * c.dn_dv;
+    if (c.q_heads * c.head_dim > kmax) kmax = c.q_heads * c.head_dim;
+    size_t smem = mk::sk::smem_bytes(mk::sk::X_NORM, mk::sk::TMAX, c.hidden, 0);
+    const size_t sg = mk::sk::smem_bytes(mk::sk::X_GATED, mk::sk::TMAX, c.dn_heads * c.dn_dv,
+                                         c.dn_dv);
+    const size_t sc = mk::sk::smem_bytes(mk::sk::X_COPY, mk::sk::TMAX, kmax, 0);
+    if (sg > smem) smem = sg;
+    if (sc > smem) smem = sc;
+    // bulk-copied operand rows start 16-byte aligned
+    const bool rows16 = c.hidden % 4 == 0 && e->lay.pw % 4 == 0 && e->lay.aw % 4 == 0 &&
+                        (c.dn_heads * c.dn_dv) % 4 == 0 && e->hm.ch % 4 == 0 && c.mlp % 8 == 0 &&
+                        (c.q_heads * c.head_dim) % 8 == 0;
+    e->sk_ok = smem <= 227u * 1024u && c.dn_dv % 32 == 0 && rows16 &&
+               cudaFuncSetAttribute(mk::sk::skinny_gemv_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    int(smem)) == cudaSuccess &&
+               cudaFuncSetAttribute(mk::vf::attn_chunk_kernel<256>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    int(mk::vf::att_smem<256>())) == cudaSuccess &&
+               cudaFuncSetAttribute(mk::vf::attn_chunk_kernel<128>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    int(mk::vf::att_smem<128>())) == cudaSuccess &&
+               cudaFuncSetAttribute(mk::vf::attn_chunk_kernel<64>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    int(mk::vf::att_smem<64>())) == cudaSuccess;
+  }
   cudaGetLastError();
   {
     const int H = c.hidden, T = lay.tmax;
@@ -827,6 +1137,7 @@ int mk_reset(mk_engine* e) {
   e->amax_toggle = 0;
   e->amax_valid = false;
   e->pending_verify = 0;
+  e->replay_n = 0;
   return MK_OK;
 }
 
@@ -895,15 +1206,25 @@ int mk_verify(mk_engine* e, const int32_t* tokens_host, int n, float* logits_out
   for (int i = 0; i < n; ++i)
     if (tokens_host[i] < 0 || tokens_host[i] >= e->cfg.vocab) return MK_ERR_ARG;
   if (e->pf_ok) {
-    // one chunk: every projection a tensor-core GEMM over the n positions,
-    // the scans writing the state after each position to its own buffer
-    for (int j = 0; j < n; ++j) e->verify_bufs[j] = (e->cur_buf + 1 + j) % mk::kStateBufs;
-    const int rc = run_chunk(e, tokens_host, n, e->verify_bufs, logits_out);
+    // one chunk: every projection one pass over its weights for the n
+    // positions; the DeltaNet layers first replay what the last accept
+    // kept, then record the chunk's positions for the next accept
+    VerifyPlan vp;
+    vp.R = e->replay_n;
+    vp.rsel = e->replay_sel;
+    vp.wsel = e->replay_sel ^ 1;
+    vp.nb = vp.R > 0 ? (e->cur_buf + 1) % mk::kStateBufs : e->cur_buf;
+    const int rc = run_chunk(e, tokens_host, n, &vp, logits_out);
     if (rc != MK_OK) return rc;
+    e->cur_buf = vp.nb;
+    e->replay_n = 0;
+    e->vlog_sel = vp.wsel;
+    e->verify_logged = true;
     e->pending_verify = n;
     e->amax_valid = false;
     return MK_OK;
   }
+  e->verify_logged = false;
   // no chunk path: one decode launch per position, each reading the state
   // after the previous position and writing its own checkpoint buffer
   int src = e->cur_buf, k = 0;
@@ -925,7 +1246,12 @@ int mk_accept(mk_engine* e, int n_keep) {
   if (!e) return MK_ERR_ARG;
   if (!e->pending_verify) return MK_ERR_STATE;
   if (n_keep < 1 || n_keep > e->pending_verify) return MK_ERR_ARG;
-  e->cur_buf = e->verify_bufs[n_keep - 1];
+  if (e->verify_logged) {
+    e->replay_n = n_keep;  // applied by the next call that reads the state
+    e->replay_sel = e->vlog_sel;
+  } else {
+    e->cur_buf = e->verify_bufs[n_keep - 1];
+  }
   e->pos += n_keep;
   e->pending_verify = 0;
   return MK_OK;
@@ -976,6 +1302,8 @@ int mk_set_state(mk_engine* e, int pos, const float* dn_state, const float* conv
 int mk_get_state(mk_engine* e, float* dn_state, float* conv_state, void* k_cache,
                  void* v_cache) {
   if (!e) return MK_ERR_ARG;
+  const int rp = replay_pending(e);
+  if (rp != MK_OK) return rp;
   const Layout& L = e->lay;
   const DevModel& m = e->hm;
   const int b = e->cur_buf;

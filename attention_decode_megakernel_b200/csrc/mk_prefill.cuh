@@ -35,12 +35,6 @@ constexpr uint32_t TILE_X_BYTES = BN * BK * 2;
 constexpr uint32_t STAGE_BYTES = TILE_W_BYTES + 2 * TILE_X_BYTES;  // W, x_hi, x_lo
 constexpr size_t GEMM_SMEM = size_t(STAGES) * STAGE_BYTES + 1024 + 256;
 
-// Per-position state copies of a verify chunk: p[t] receives the state after
-// position t (p[0] == nullptr: a prompt chunk, the state is updated in place).
-struct Ckpt {
-  float* p[kMaxVerify];
-};
-
 struct GemmArgs {
   CUtensorMap tw;    // weights [n_out][K] bf16, box {BK, BM}
   CUtensorMap tx;    // activations [2][x_lo_row][K] bf16 (hi rows, then lo rows), box {BK, BN}
@@ -330,6 +324,7 @@ __device__ __forceinline__ void store_split(uint16_t* p, size_t lo, float v) {
 
 // x[t] = embedding row of tokens[t] (fp32)
 __global__ void embed_kernel(const int32_t* tokens, const uint16_t* E, float* X, int H) {
+  griddep_launch_dependents();
   const int t = blockIdx.x;
   const uint16_t* row = E + size_t(tokens[t]) * H;
   for (int i = threadIdx.x; i < H; i += blockDim.x) X[size_t(t) * H + i] = bf2f(row[i]);
@@ -351,15 +346,14 @@ __global__ void rmsnorm_bf16_kernel(const float* X, const uint16_t* gain, uint16
 // Causal depthwise conv + SiLU over T positions, one thread per (position,
 // channel): Cv[t][c] = SiLU(w0 u_{t-3} + w1 u_{t-2} + w2 u_{t-1} + w3 u_t)
 // with u = the raw in-projection columns of P and u_{<0} taken from the
-// carried history `state` = (u_{-3}, u_{-2}, u_{-1}).  With checkpoints the
-// history after position t, (u_{t-2}, u_{t-1}, u_t), goes to ck.p[t].
+// carried history `state` = (u_{-3}, u_{-2}, u_{-1}).
 __device__ __forceinline__ float conv_input(const float* P, int ldp, const float4& s, int t,
                                             int c) {
   return t >= 0 ? P[size_t(t) * ldp + c] : (t == -1 ? s.z : t == -2 ? s.y : s.x);
 }
 
 __global__ void conv_kernel(const float* P, int ldp, const float4* state, const uint16_t* conv_w,
-                            int ch, float* Cv, int ldc, Ckpt ck) {
+                            int ch, float* Cv, int ldc) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x, t = blockIdx.y;
   if (c >= ch) return;
   const float4 s = state[c];
@@ -368,7 +362,6 @@ __global__ void conv_kernel(const float* P, int ldp, const float4* state, const 
   const float u1 = conv_input(P, ldp, s, t - 1, c), u0 = P[size_t(t) * ldp + c];
   const float y = bf_lo(wc.x) * u3 + bf_hi(wc.x) * u2 + bf_lo(wc.y) * u1 + bf_hi(wc.y) * u0;
   Cv[size_t(t) * ldc + c] = siluf_(y);
-  if (ck.p[0]) reinterpret_cast<float4*>(ck.p[t])[c] = make_float4(u2, u1, u0, 0.f);
 }
 
 // The carried history after T positions (a separate launch: every conv
@@ -407,95 +400,6 @@ __global__ void dn_prep_kernel(const float* Cv, int ldc, const float* P, int ldp
   }
 }
 
-// Gated delta rule over T positions, the state rows in registers: each
-// warp owns RPW = 2 rows of one head (lane: DK/32 entries of a row), a block
-// 8 warps = 16 rows.  The block stages REC_TT positions of q, k, gates and
-// its v values in shared memory, then steps through them:
-//   u = beta (v - alpha S.k),  S <- alpha S + u k^T,  o = S.q = alpha S_old.q + u (k.q)
-// The four dot products of a step (S.k and S.q of both rows) share one
-// shuffle tree.  CKPT: the state after position t goes to ck.p[t] and S is
-// left as it was (verify); otherwise S is updated in place.
-constexpr int REC_WARPS = 8;
-constexpr int REC_RPW = 2;
-constexpr int REC_TT = 32;
-template <int DK, bool CKPT>
-__global__ void __launch_bounds__(REC_WARPS * 32) recurrence_kernel(
-    float* S, const float* QK, const float4* BAK, const float* Cv, int ldc, int vcol, float* O,
-    int ldo, int T, Ckpt ck) {
-  constexpr int EPL = DK / 32;
-  constexpr int BR = REC_WARPS * REC_RPW;  // rows per block
-  __shared__ __align__(16) float sqk[REC_TT][2 * DK];
-  __shared__ float4 sgate[REC_TT];
-  __shared__ float sv[REC_TT][BR];
-  const int h = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int brow0 = blockIdx.y * BR;          // first row of the block within the head
-  const int row0 = brow0 + warp * REC_RPW;    // value coordinate i of this warp's first row
-  float st[REC_RPW][EPL];
-#pragma unroll
-  for (int r = 0; r < REC_RPW; ++r)
-#pragma unroll
-    for (int e = 0; e < EPL; ++e)
-      st[r][e] = S[(size_t(h) * DK + row0 + r) * DK + lane * EPL + e];
-  const float* qk = QK + size_t(h) * T * 2 * DK;
-  const float4* bak = BAK + size_t(h) * T;
-  const float* vsrc = Cv + vcol + h * DK + brow0;
-  for (int t0 = 0; t0 < T; t0 += REC_TT) {
-    const int nt = min(REC_TT, T - t0);
-    __syncthreads();  // the previous tile is consumed
-    const float4* src4 = reinterpret_cast<const float4*>(qk + size_t(t0) * 2 * DK);
-    for (int i = threadIdx.x; i < nt * (2 * DK / 4); i += blockDim.x)
-      reinterpret_cast<float4*>(&sqk[0][0])[i] = src4[i];
-    for (int i = threadIdx.x; i < nt; i += blockDim.x) sgate[i] = bak[t0 + i];
-    for (int i = threadIdx.x; i < nt * BR; i += blockDim.x)
-      sv[i / BR][i % BR] = vsrc[size_t(t0 + i / BR) * ldc + (i % BR)];
-    __syncthreads();
-    for (int tt = 0; tt < nt; ++tt) {
-      float q[EPL], k[EPL];
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        q[e] = sqk[tt][lane * EPL + e];
-        k[e] = sqk[tt][DK + lane * EPL + e];
-      }
-      const float4 g = sgate[tt];  // {beta, alpha, k.q, -}
-      float pk0 = 0.f, pq0 = 0.f, pk1 = 0.f, pq1 = 0.f;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        pk0 = fmaf(st[0][e], k[e], pk0);
-        pq0 = fmaf(st[0][e], q[e], pq0);
-        pk1 = fmaf(st[1][e], k[e], pk1);
-        pq1 = fmaf(st[1][e], q[e], pq1);
-      }
-      // lanes 0-7: S0.k, 8-15: S0.q, 16-23: S1.k, 24-31: S1.q
-      const float z = reduce4(pk0, pq0, pk1, pq1, lane);
-      const float sk0 = __shfl_sync(0xffffffffu, z, 0), sk1 = __shfl_sync(0xffffffffu, z, 16);
-      const float u0 = g.x * (sv[tt][warp * REC_RPW] - g.y * sk0);
-      const float u1 = g.x * (sv[tt][warp * REC_RPW + 1] - g.y * sk1);
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        st[0][e] = fmaf(g.y, st[0][e], u0 * k[e]);
-        st[1][e] = fmaf(g.y, st[1][e], u1 * k[e]);
-      }
-      if (lane == 8) O[size_t(t0 + tt) * ldo + h * DK + row0] = fmaf(g.y, z, u0 * g.z);
-      if (lane == 24) O[size_t(t0 + tt) * ldo + h * DK + row0 + 1] = fmaf(g.y, z, u1 * g.z);
-      if constexpr (CKPT) {
-#pragma unroll
-        for (int r = 0; r < REC_RPW; ++r)
-#pragma unroll
-          for (int e = 0; e < EPL; ++e)
-            ck.p[t0 + tt][(size_t(h) * DK + row0 + r) * DK + lane * EPL + e] = st[r][e];
-      }
-    }
-  }
-  if constexpr (!CKPT) {
-#pragma unroll
-    for (int r = 0; r < REC_RPW; ++r)
-#pragma unroll
-      for (int e = 0; e < EPL; ++e)
-        S[(size_t(h) * DK + row0 + r) * DK + lane * EPL + e] = st[r][e];
-  }
-}
-
 // G[t][h*dv + i] = split(RMSNorm_dv(O[t][h]) * w_i * SiLU(z[t][h*dv+i]))
 __global__ void gated_norm_kernel(const float* O, int ldo, const float* P, int ldp, int zcol,
                                   const uint16_t* w, uint16_t* G, int ldg, float eps, size_t lo) {
@@ -519,6 +423,8 @@ __global__ void swiglu_kernel(const float* P, int ldp, int I, uint16_t* Hb, int 
 // into the bf16 cache.  grid (T, nq + nkv), blockDim = hd / 2.
 __global__ void rope_kv_kernel(float* P, int ldp, int nq, int nkv, int hd, uint16_t* kc,
                                uint16_t* vc, int max_ctx, int pos0, float theta) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int t = blockIdx.x, hh = blockIdx.y, i = threadIdx.x, half = hd / 2;
   const int pos = pos0 + t;
   const double inv_freq = pow(double(theta), -2.0 * double(i) / double(hd));
@@ -689,7 +595,8 @@ __global__ void __launch_bounds__(ATT_SPLIT_WARPS * 32) attn_split_kernel(
 // bf16 operands for the output-projection GEMM.  grid (nq, T), HD threads.
 template <int HD>
 __global__ void attn_merge_kernel(const float* part, int nq, int nsplit, uint16_t* Ob, int ldob,
-                                  size_t lo) {
+                                  size_t lo, float* Of) {
+  griddep_launch_dependents();
   const int h = blockIdx.x, t = blockIdx.y, i = threadIdx.x;
   const float* base = part + (size_t(t) * nq + h) * nsplit * (HD + 2);
   float M = -INFINITY;
@@ -704,7 +611,10 @@ __global__ void attn_merge_kernel(const float* part, int nq, int nsplit, uint16_
       num = fmaf(wgt, ps[i], num);
     }
   }
-  store_split(Ob + size_t(t) * ldob + h * HD + i, lo, num / den);
+  if (Of)
+    Of[size_t(t) * ldob + h * HD + i] = num / den;  // fp32 rows of the same width
+  else
+    store_split(Ob + size_t(t) * ldob + h * HD + i, lo, num / den);
 }
 
 }  // namespace pf

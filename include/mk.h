@@ -105,7 +105,7 @@ typedef struct {
 typedef struct mk_engine mk_engine;
 
 /* Bytes of device workspace mk_create needs for this config (recurrent
- * state, verify checkpoints, KV cache, activations, exchange words, and the
+ * state buffers, verify records, KV cache, activations, exchange words, and the
  * decode kernel's copies of the layer weights, see mk_create).
  * Returns 0 for an invalid config. */
 size_t mk_workspace_bytes(const mk_config *cfg);
@@ -183,27 +183,33 @@ int mk_generate(mk_engine *e, int32_t first_token, int n, int32_t *tokens_out,
 
 /* Verify n tokens at once (1 <= n <= max_verify), the speculative-decoding
  * shape (several draft tokens checked by one forward pass, with the
- * recurrent state checkpointed for rollback; the follow-up post
+ * recurrent state kept recoverable for rollback; the follow-up post
  * "업데이트: 단일 RTX 3090에서 Qwen 3.8 27B를 140 tok/s로 구동 (Megakernel:
  * KL divergence", speed list: four draft tokens checked for the cost of one
  * forward pass, greedy output unchanged): the stack runs over positions
- * pos .. pos+n-1 as one chunk -- every projection one tensor-core GEMM with
- * M = n (weights read once for the n positions), the conv and the gated
- * delta rule advanced position by position -- and writes the logits of
- * every position to logits_out (device, float32 [n][vocab], not NULL), the
- * DeltaNet and conv state after each position to its own checkpoint buffer,
- * and K/V of the n positions to the cache.  Results equal n decode steps up
- * to rounding.  The current state is left as it was; the position does not
- * advance until mk_accept.  MK_ERR_STATE while a verify is pending. */
+ * pos .. pos+n-1 as one chunk -- every projection one pass over its weights
+ * for the n positions, the conv and the gated delta rule advanced position
+ * by position -- and writes the logits of every position to logits_out
+ * (device, float32 [n][vocab], not NULL) and K/V of the n positions to the
+ * cache.  Instead of the state after every position it records, per
+ * DeltaNet layer and position, the normalised key, the value, alpha, beta
+ * and the conv inputs (a few KB).  Positions kept by the previous
+ * mk_accept are applied to the state first, inside this call.  Results
+ * equal n decode steps up to rounding.  The position does not advance until
+ * mk_accept.  MK_ERR_STATE while a verify is pending. */
 int mk_verify(mk_engine *e, const int32_t *tokens_host, int n,
               float *logits_out);
 
-/* Keep the first n_keep (1..n) positions of the last mk_verify: the state
- * becomes the checkpoint after position n_keep-1 and the position advances
- * by n_keep (the rollback of rejected draft tokens that exact greedy
- * speculative decoding needs; same follow-up post, accuracy paragraph:
- * greedy output stays the main model's greedy choice).
- * MK_ERR_STATE if no verify is pending. */
+/* Keep the first n_keep (1..n) positions of the last mk_verify and advance
+ * the position by n_keep (the rollback of rejected draft tokens that exact
+ * greedy speculative decoding needs; same follow-up post, accuracy
+ * paragraph: greedy output stays the main model's greedy choice).  No work
+ * is launched: the next call that reads the state (verify, decode,
+ * generate, prefill, mk_get_state) first replays the n_keep recorded
+ * positions on it, so the state after a rejected position is never
+ * written.  (Without the chunk path, mk_verify falls back to one decode
+ * launch per position with a full state copy after each, and mk_accept
+ * selects the copy.)  MK_ERR_STATE if no verify is pending. */
 int mk_accept(mk_engine *e, int n_keep);
 
 /* Current position (number of tokens consumed). */

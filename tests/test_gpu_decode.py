@@ -239,8 +239,9 @@ def test_verify_against_oracle_then_accept(mk, cfg_name, keep):
 
 
 def test_verify_twice_and_cycle_buffers(mk):
-    """Repeated verify/accept cycles walk the checkpoint buffers round the
-    ring; the result tracks the oracle."""
+    """Repeated verify/accept cycles: each verify first replays the
+    positions the previous accept kept, then records its own; the state
+    buffers rotate; the result tracks the oracle."""
     cfg = synth.tiny_config(max_ctx=256)
     w = synth.make_weights(cfg)
     eng = mk.Engine(cfg, w)
@@ -265,6 +266,66 @@ def test_verify_twice_and_cycle_buffers(mk):
         eng.accept(keep)
         for j in range(keep):
             orc.step(int(toks[j]))
+    _check_state(eng, orc)
+    print(tr.finish())
+
+
+def test_accepted_positions_replayed_by_every_kind_of_call(mk):
+    """After mk_accept the kept positions are applied by whichever call reads
+    the state next: a prompt chunk, a verify, a decode step or generate.
+    Logits of every call track the oracle fed the same accepted tokens."""
+    cfg = synth.tiny_config(max_ctx=256)
+    w = synth.make_weights(cfg)
+    eng = mk.Engine(cfg, w)
+    orc = oracle.OracleModel(cfg, w)
+    tr = Tracker()
+    rng = np.random.default_rng(23)
+    logits = torch.empty(cfg.vocab, dtype=torch.float32, device="cuda")
+    vl = torch.empty((8, cfg.vocab), dtype=torch.float32, device="cuda")
+
+    def verify_accept(n, keep):
+        toks = rng.integers(0, cfg.vocab, n)
+        eng.verify(toks, vl[:n])
+        eng.sync()
+        ref_orc = orc.clone()
+        for j in range(n):
+            ref, _ = ref_orc.step(int(toks[j]))
+            tr.logits(_np(vl[j]), ref)
+        eng.accept(keep)
+        for j in range(keep):
+            orc.step(int(toks[j]))
+
+    prompt = synth.make_tokens(cfg.vocab, 16)
+    eng.prefill(prompt)
+    for t in prompt:
+        orc.step(int(t))
+    verify_accept(5, 2)
+    more = rng.integers(0, cfg.vocab, 12)  # a prompt chunk reads the state next
+    eng.prefill(more, logits)
+    for t in more:
+        ref, _ = orc.step(int(t))
+    eng.sync()
+    tr.logits(_np(logits), ref)
+    verify_accept(6, 6)
+    verify_accept(3, 1)  # a verify replays the 6 kept above
+    tok = int(rng.integers(0, cfg.vocab))
+    eng.decode_step(tok, logits)  # a decode step replays the 1 kept above
+    ref, _ = orc.step(tok)
+    eng.sync()
+    tr.logits(_np(logits), ref)
+    verify_accept(4, 3)
+    n = 4
+    toks = torch.zeros(n, dtype=torch.int32, device="cuda")
+    lg = torch.empty((n, cfg.vocab), dtype=torch.float32, device="cuda")
+    first = int(rng.integers(0, cfg.vocab))
+    eng.generate(first, n, toks, lg)  # generate replays the 3 kept above
+    eng.sync()
+    fed = first
+    for i in range(n):
+        ref, _ = orc.step(fed)
+        tr.logits(_np(lg[i]), ref)
+        fed = int(_np(toks)[i])
+    assert eng.position == orc.pos
     _check_state(eng, orc)
     print(tr.finish())
 
