@@ -408,8 +408,37 @@ int launch_skinny(mk_engine* e, mk::sk::Args a) {
   const int rpb = (mk::sk::WARPS / a.kw) * mk::sk::RW;
   const int lpb = a.pair ? rpb / 2 : rpb;
   const int nblk = (a.N + lpb - 1) / lpb;
-  return launch_pdl(e, mk::sk::skinny_gemv_kernel, dim3(nblk < mk::sk::MAX_CTAS ? nblk : mk::sk::MAX_CTAS),
-                    dim3(mk::sk::THREADS), mk::sk::smem_bytes(a.mode, a.T, a.K, a.dv), a);
+  const dim3 grid(nblk < mk::sk::MAX_CTAS ? nblk : mk::sk::MAX_CTAS), block(mk::sk::THREADS);
+  const size_t smem = mk::sk::smem_bytes(a.mode, a.T, a.K, a.dv);
+  switch (a.T) {
+    case 1: return launch_pdl(e, mk::sk::skinny_gemv_kernel<1>, grid, block, smem, a);
+    case 2: return launch_pdl(e, mk::sk::skinny_gemv_kernel<2>, grid, block, smem, a);
+    case 3: return launch_pdl(e, mk::sk::skinny_gemv_kernel<3>, grid, block, smem, a);
+    case 4: return launch_pdl(e, mk::sk::skinny_gemv_kernel<4>, grid, block, smem, a);
+    case 5: return launch_pdl(e, mk::sk::skinny_gemv_kernel<5>, grid, block, smem, a);
+    case 6: return launch_pdl(e, mk::sk::skinny_gemv_kernel<6>, grid, block, smem, a);
+    case 7: return launch_pdl(e, mk::sk::skinny_gemv_kernel<7>, grid, block, smem, a);
+    case 8: return launch_pdl(e, mk::sk::skinny_gemv_kernel<8>, grid, block, smem, a);
+  }
+  return MK_ERR_ARG;
+}
+
+// Largest dynamic shared memory of every skinny instantiation.
+bool skinny_attrs(size_t smem) {
+  const void* fns[8] = {
+      reinterpret_cast<const void*>(mk::sk::skinny_gemv_kernel<1>),
+      reinterpret_cast<const void*>(mk::sk::skinny_gemv_kernel<2>),
+      reinterpret_cast<const void*>(mk::sk::skinny_gemv_kernel<3>),
+      reinterpret_cast<const void*>(mk::sk::skinny_gemv_kernel<4>),
+      reinterpret_cast<const void*>(mk::sk::skinny_gemv_kernel<5>),
+      reinterpret_cast<const void*>(mk::sk::skinny_gemv_kernel<6>),
+      reinterpret_cast<const void*>(mk::sk::skinny_gemv_kernel<7>),
+      reinterpret_cast<const void*>(mk::sk::skinny_gemv_kernel<8>)};
+  for (const void* f : fns)
+    if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+      return false;
+  return true;
 }
 
 // Record set `sel` of DeltaNet layer `sub`.
@@ -1064,10 +1093,7 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
     const bool rows16 = c.hidden % 4 == 0 && e->lay.pw % 4 == 0 && e->lay.aw % 4 == 0 &&
                         (c.dn_heads * c.dn_dv) % 4 == 0 && e->hm.ch % 4 == 0 && c.mlp % 8 == 0 &&
                         (c.q_heads * c.head_dim) % 8 == 0;
-    e->sk_ok = smem <= 227u * 1024u && c.dn_dv % 32 == 0 && rows16 &&
-               cudaFuncSetAttribute(mk::sk::skinny_gemv_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    int(smem)) == cudaSuccess &&
+    e->sk_ok = smem <= 227u * 1024u && c.dn_dv % 32 == 0 && rows16 && skinny_attrs(smem) &&
                cudaFuncSetAttribute(mk::vf::attn_chunk_kernel<256>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     int(mk::vf::att_smem<256>())) == cudaSuccess &&

@@ -137,6 +137,18 @@ __device__ __forceinline__ bool named_sync_or(int id, int nthreads, bool pred) {
 // ---- numerics -------------------------------------------------------------------
 __device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+// {a, b} += {x0, x1} * {y0, y1}: one packed fp32 FMA instruction (two
+// round-to-nearest fmaf, the same results as two separate ones).
+__device__ __forceinline__ void ffma2(float& a, float& b, float x0, float x1, float y0, float y1) {
+  asm("{\n\t.reg .b64 c, x, y;\n\t"
+      "mov.b64 c, {%0, %1};\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 y, {%4, %5};\n\t"
+      "fma.rn.f32x2 c, x, y, c;\n\t"
+      "mov.b64 {%0, %1}, c;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "f"(x0), "f"(x1), "f"(y0), "f"(y1));
+}
 __device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
 // float -> bf16 bits, round to nearest even (finite inputs).
 __device__ __forceinline__ uint16_t f2bf(float f) {

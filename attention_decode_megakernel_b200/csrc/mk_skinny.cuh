@@ -92,11 +92,15 @@ __device__ __forceinline__ void rows_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-constexpr int VL = 4;  // 8-byte vectors of a row in flight per lane
+// 8-byte vectors of a row in flight per lane (fewer with more tokens: the
+// accumulators take the registers)
+constexpr int vl_for(int T) { return T <= 5 ? 4 : 2; }
 
-// acc[q][t] += sum_e w_q[e] * x_t[e] over one 8-byte vector of each row
-__device__ __forceinline__ void fma_vec(float (&acc)[RW][TMAX], const uint2 (&u)[RW],
-                                        const float* xs, int K, int T, int v) {
+// {a0, a1}[q][t] += the even / odd products of one 8-byte vector of row q with
+// x_t, two at a time (packed fp32 FMA)
+template <int T>
+__device__ __forceinline__ void fma_vec(float (&a0)[RW][T], float (&a1)[RW][T],
+                                        const uint2 (&u)[RW], const float* xs, int K, int v) {
   float w[RW][4];
 #pragma unroll
   for (int q = 0; q < RW; ++q) {
@@ -104,21 +108,21 @@ __device__ __forceinline__ void fma_vec(float (&acc)[RW][TMAX], const uint2 (&u)
     w[q][2] = bfl(u[q].y); w[q][3] = bfh(u[q].y);
   }
 #pragma unroll
-  for (int t = 0; t < TMAX; ++t) {
-    if (t < T) {
-      const float4 p = reinterpret_cast<const float4*>(xs + t * K)[v];
+  for (int t = 0; t < T; ++t) {
+    const float4 p = reinterpret_cast<const float4*>(xs + t * K)[v];
 #pragma unroll
-      for (int q = 0; q < RW; ++q) {
-        acc[q][t] = fmaf(w[q][0], p.x, acc[q][t]);
-        acc[q][t] = fmaf(w[q][1], p.y, acc[q][t]);
-        acc[q][t] = fmaf(w[q][2], p.z, acc[q][t]);
-        acc[q][t] = fmaf(w[q][3], p.w, acc[q][t]);
-      }
+    for (int q = 0; q < RW; ++q) {
+      ffma2(a0[q][t], a1[q][t], w[q][0], w[q][1], p.x, p.y);
+      ffma2(a0[q][t], a1[q][t], w[q][2], w[q][3], p.z, p.w);
     }
   }
 }
 
+// T == a.T: one instantiation per token count, so only live accumulators
+// take registers.
+template <int T>
 __global__ void __launch_bounds__(THREADS, 2) skinny_gemv_kernel(const __grid_constant__ Args a) {
+  constexpr int VL = vl_for(T);
   extern __shared__ __align__(16) float xs[];  // [T][K] x rows, then z rows, then gain
   __shared__ float red[2][WARPS][32];
   __shared__ float inv_s[TMAX];
@@ -126,7 +130,7 @@ __global__ void __launch_bounds__(THREADS, 2) skinny_gemv_kernel(const __grid_co
   __shared__ int bad;
   griddep_launch_dependents();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int T = a.T, K = a.K;
+  const int K = a.K;
   const bool gated = a.mode == X_GATED;
   float* zs = xs + T * K;
   float* gs = xs + T * K * (gated ? 2 : 1);
@@ -253,11 +257,11 @@ __global__ void __launch_bounds__(THREADS, 2) skinny_gemv_kernel(const __grid_co
     const uint2* wr[RW];
 #pragma unroll
     for (int q = 0; q < RW; ++q) wr[q] = row_ptr(blk, q);
-    float acc[RW][TMAX];
+    float a0[RW][T], a1[RW][T];
 #pragma unroll
     for (int q = 0; q < RW; ++q)
 #pragma unroll
-      for (int t = 0; t < TMAX; ++t) acc[q][t] = 0.f;
+      for (int t = 0; t < T; ++t) a0[q][t] = a1[q][t] = 0.f;
     for (int v = v0 + lane; v < v1; v += 32 * VL) {
       if (!first) {
 #pragma unroll
@@ -270,12 +274,16 @@ __global__ void __launch_bounds__(THREADS, 2) skinny_gemv_kernel(const __grid_co
       first = false;
 #pragma unroll
       for (int i = 0; i < VL; ++i)
-        if (v + 32 * i < v1) fma_vec(acc, u[i], xs, K, T, v + 32 * i);
+        if (v + 32 * i < v1) fma_vec<T>(a0, a1, u[i], xs, K, v + 32 * i);
     }
     first = false;
     // butterfly: after five exchanges lane j holds the warp's sum of value
     // j = q * TMAX + t
-    float* val = &acc[0][0];
+    float val[RW * TMAX];
+#pragma unroll
+    for (int q = 0; q < RW; ++q)
+#pragma unroll
+      for (int t = 0; t < TMAX; ++t) val[q * TMAX + t] = t < T ? a0[q][t] + a1[q][t] : 0.f;
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) {
       const bool up = lane & o;
