@@ -1090,7 +1090,7 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
     if (sg > smem) smem = sg;
     if (sc > smem) smem = sc;
     // bulk-copied operand rows start 16-byte aligned
-    const bool rows16 = c.hidden % 4 == 0 && e->lay.pw % 4 == 0 && e->lay.aw % 4 == 0 &&
+    const bool rows16 = c.hidden % 128 == 0 && c.hidden <= 4096 && e->lay.pw % 4 == 0 && e->lay.aw % 4 == 0 &&
                         (c.dn_heads * c.dn_dv) % 4 == 0 && e->hm.ch % 4 == 0 && c.mlp % 8 == 0 &&
                         (c.q_heads * c.head_dim) % 8 == 0;
     e->sk_ok = smem <= 227u * 1024u && c.dn_dv % 32 == 0 && rows16 && skinny_attrs(smem) &&

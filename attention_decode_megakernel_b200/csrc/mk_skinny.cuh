@@ -46,7 +46,7 @@ struct Args {
   int kw;              // warps splitting one row block's K range (1, 2, 4 or 8)
   int mode;            // Prologue
   int pair;            // C[t][j] = SiLU(W0[j] . x_t) * (W1[j] . x_t)
-  // X_NORM: x = X[t][k] * rsqrt(mean_k X[t]^2 + eps) * gain[k]
+  // X_NORM: x = X[t][k] * rsqrt(mean_k X[t]^2 + eps) * gain[k]  (K % 128 == 0)
   // X_COPY: x = X[t][k]
   // X_GATED: x = O[t][c] * rsqrt(mean over c's head of O^2 + eps) *
   //          gain[c % dv] * SiLU(X2[t][c])       (O = X, z = X2)
@@ -126,6 +126,7 @@ __global__ void __launch_bounds__(THREADS, 2) skinny_gemv_kernel(const __grid_co
   extern __shared__ __align__(16) float xs[];  // [T][K] x rows, then z rows, then gain
   __shared__ float red[2][WARPS][32];
   __shared__ float inv_s[TMAX];
+  __shared__ float ssp[TMAX][32];  // X_NORM: sums of squares of 128-element pieces
   __shared__ __align__(8) uint64_t bar;
   __shared__ int bad;
   griddep_launch_dependents();
@@ -208,27 +209,28 @@ __global__ void __launch_bounds__(THREADS, 2) skinny_gemv_kernel(const __grid_co
     return;
   }
   if (a.mode == X_NORM) {
-    if (warp < T) {
-      float s = 0.f;
-      for (int k = lane * 4; k < K; k += 128) {
-        const float4 v = *reinterpret_cast<const float4*>(xs + warp * K + k);
-        s = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, s))));
-      }
-      s = warp_sum(s);
-      if (lane == 0) inv_s[warp] = 1.0f / sqrtf(s / float(K) + a.eps);
-    }
-    __syncthreads();
+    // x * gain in place, and the sums of squares of x in 128-element pieces
+    // (K a multiple of 128: a warp's 32 float4 never straddle two rows); the
+    // factor rsqrt(mean x^2 + eps) multiplies the dot products at the end
     const int k4 = K / 4;
     for (int i = tid; i < T * k4; i += THREADS) {
-      const int t = i / k4;
+      const int t = i / k4, kk = i - t * k4;
       float4 v = reinterpret_cast<float4*>(xs)[i];
-      const float4 gk = reinterpret_cast<const float4*>(gs)[i - t * k4];
-      const float r = inv_s[t];
-      v.x = v.x * r * gk.x;
-      v.y = v.y * r * gk.y;
-      v.z = v.z * r * gk.z;
-      v.w = v.w * r * gk.w;
+      const float4 gk = reinterpret_cast<const float4*>(gs)[kk];
+      float s = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, v.w * v.w)));
+      s = warp_sum(s);
+      if (lane == 0) ssp[t][kk >> 5] = s;
+      v.x *= gk.x;
+      v.y *= gk.y;
+      v.z *= gk.z;
+      v.w *= gk.w;
       reinterpret_cast<float4*>(xs)[i] = v;
+    }
+    __syncthreads();
+    if (tid < T) {
+      float tot = 0.f;
+      for (int c = 0; c < (k4 >> 5); ++c) tot += ssp[tid][c];
+      inv_s[tid] = 1.0f / sqrtf(tot / float(K) + a.eps);
     }
   } else if (gated) {
     // one warp per (token, head); dv a multiple of 32
@@ -300,6 +302,7 @@ __global__ void __launch_bounds__(THREADS, 2) skinny_gemv_kernel(const __grid_co
       const int gg = tid >> 5, j = tid & 31, q = j / TMAX, t = j % TMAX;
       float s = 0.f;
       for (int p = 0; p < kw; ++p) s += red[par][gg * kw + p][j];
+      if (a.mode == X_NORM && t < T) s *= inv_s[t];
       if (a.pair) {
         // rows q (gate) and q + 1 (up) of the same output j; q even
         const float upv = __shfl_down_sync(0xffffffffu, s, TMAX);
