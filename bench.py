@@ -30,7 +30,7 @@ GEN = 128
 # DRAM bytes (read + written) of one decode launch at context 520, from an ncu
 # capture of the current decode kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum); None once the kernel changes.
-DECODE_TRAFFIC_BYTES = None
+DECODE_TRAFFIC_BYTES = 1340556000  # 1.311269 GB read + 29.286912 MB written
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
@@ -481,7 +481,15 @@ def extra_workloads(mk, synth, torch, np, prefill_ms_per_call, hbm, tc_peak, pea
     dn = cfg.n_dn * cfg.dn_heads * cfg.dn_dv * cfg.dn_dk * 4
     conv = cfg.n_dn * cfg.conv_channels * (cfg.conv_k - 1) * 4
     kvb = cfg.n_attn * 2 * cfg.kv_heads * cfg.head_dim * 2
-    vbytes = weights + dn + conv + 5 * (dn + conv) + kvb * (ctx + 100) + 5 * kvb + 5 * cfg.vocab * 4
+    # per DeltaNet layer and position: key, value, alpha, beta, conv inputs
+    rec = cfg.n_dn * (cfg.dn_heads * (cfg.dn_dk + cfg.dn_dv + 2) + cfg.conv_channels) * 4
+    acc = kept / calls
+    # weights once; the state read and written once (the previous accept's
+    # positions replayed into the next buffer); 5 records written and the
+    # accepted ones read back; KV read over the context and 5 positions
+    # appended; 5 rows of logits
+    vbytes = (weights + 2 * (dn + conv) + 5 * rec + acc * rec + kvb * (ctx + 100) + 5 * kvb
+              + 5 * cfg.vocab * 4)
     out["verify_5tok_ctx4096"] = {
         "calls_s": calls / (dev_ms / 1000.0), "ms_per_call": dev_ms / calls,
         "positions_s": 5 * calls / (dev_ms / 1000.0), "accepted_per_call": kept / calls,

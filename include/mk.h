@@ -133,7 +133,8 @@ int mk_create(const mk_config *cfg, const mk_weights *w, void *workspace,
 void mk_destroy(mk_engine *e);
 
 /* Zero the DeltaNet and conv states, empty the KV cache, clear a device
- * error and any pending verify: the start of a new sequence (launch post,
+ * error, any pending verify and any accepted positions not yet replayed:
+ * the start of a new sequence (launch post,
  * "Why nobody had done this yet?": the DeltaNet layers carry a recurrent
  * state and the attention layers a KV cache from token to token).  Weights
  * are untouched. */
