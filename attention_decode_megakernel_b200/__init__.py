@@ -93,6 +93,8 @@ def lib():
                                            C.c_int, C.c_int, vp, sz, vp]),
             "mk_debug_gemm": (C.c_int, [vp, vp, vp, C.c_int, C.c_int, C.c_int, vp]),
             "mk_debug_gemm_noalloc": (C.c_int, [vp, vp, vp, C.c_int, C.c_int, C.c_int, vp]),
+            "mk_quantize_w4": (C.c_int, [vp, C.c_int, C.c_int, vp, vp, vp]),
+            "mk_gemv_w4": (C.c_int, [vp, vp, vp, C.c_int, C.c_int, C.c_int, vp, vp]),
             "mk_strerror": (C.c_char_p, [C.c_int]),
         }
         for name, (res, args) in sig.items():
@@ -320,3 +322,26 @@ def mk_debug_gemm_noalloc(W, X, Cout, stream=None):
     st = stream if stream is not None else 0
     _check(lib().mk_debug_gemm_noalloc(_ptr(W), _ptr(X), _ptr(Cout), int(n_out), int(T), int(K),
                                        st), "mk_debug_gemm_noalloc")
+
+
+def quantize_w4(W, codes, scales, stream=None):
+    """4-bit group-wise quantisation of W (bf16 bits [rows][cols] as an int16
+    device tensor) into codes (uint8 [rows][cols / 2]) and scales (float32
+    [rows][cols / 64]), device tensors the caller provides."""
+    rows, cols = W.shape
+    if codes.numel() != rows * cols // 2 or scales.numel() != rows * cols // 64:
+        raise ValueError("codes must hold [rows][cols/2] bytes, scales [rows][cols/64] floats")
+    st = stream if stream is not None else 0
+    _check(lib().mk_quantize_w4(_ptr(W), int(rows), int(cols), _ptr(codes), _ptr(scales), st),
+           "mk_quantize_w4")
+
+
+def gemv_w4(codes, scales, x, y, stream=None):
+    """y [T][rows] = x [T][cols] times the dequantised 4-bit weights, transposed."""
+    T, cols = x.shape
+    rows = codes.numel() * 2 // cols
+    if y.numel() != T * rows or scales.numel() != rows * cols // 64:
+        raise ValueError("y must hold [T][rows] floats and scales [rows][cols/64]")
+    st = stream if stream is not None else 0
+    _check(lib().mk_gemv_w4(_ptr(codes), _ptr(scales), _ptr(x), int(T), int(rows), int(cols),
+                            _ptr(y), st), "mk_gemv_w4")

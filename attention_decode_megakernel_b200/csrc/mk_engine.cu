@@ -15,6 +15,7 @@
 #include "mk_model.cuh"
 #include "mk_prefill.cuh"
 #include "mk_skinny.cuh"
+#include "mk_lowbit.cuh"
 #include "mk_verify.cuh"
 
 namespace {
@@ -1571,6 +1572,69 @@ int mk_debug_gemm_noalloc(const void* W, const void* X, float* C, int n_out, int
   const int rblocks = int((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
   mk::pf::splitk_reduce_kernel<<<rblocks, 256, 0, st>>>(g_partial_addr[dev], ks, n, C,
                                                         g_err_addr[dev]);
+  return cuda_status(cudaGetLastError());
+}
+
+int mk_quantize_w4(const void* W, int rows, int cols, void* codes, float* scales, void* stream) {
+  if (!W || !codes || !scales || rows <= 0 || cols <= 0 || cols % mk::q4::G) return MK_ERR_ARG;
+  if (!aligned16(W) || !aligned16(codes) || !aligned16(scales)) return MK_ERR_ARG;
+  const size_t groups = size_t(rows) * (cols / mk::q4::G);
+  const size_t blocks = (groups + 255) / 256;
+  if (blocks > 0x7FFFFFFFu) return MK_ERR_UNSUPPORTED;
+  mk::q4::quantize_w4_kernel<<<unsigned(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(W), rows, cols, static_cast<uint8_t*>(codes), scales);
+  return cuda_status(cudaGetLastError());
+}
+
+int mk_gemv_w4(const void* codes, const float* scales, const float* x, int T, int rows, int cols,
+               float* y, void* stream) {
+  if (!codes || !scales || !x || !y || T < 1 || T > mk::q4::TMAX || rows <= 0 || cols <= 0 ||
+      cols % mk::q4::G)
+    return MK_ERR_ARG;
+  if (!aligned16(codes) || !aligned16(x) || (reinterpret_cast<uintptr_t>(scales) & 3u) ||
+      (reinterpret_cast<uintptr_t>(y) & 3u))
+    return MK_ERR_ARG;
+  const size_t smem = size_t(T) * cols * 4;  // the T activation rows
+  if (smem > 220u * 1024u) return MK_ERR_UNSUPPORTED;
+  int dev = 0;
+  cudaError_t r = cudaGetDevice(&dev);
+  if (r != cudaSuccess) return cuda_status(r);
+  // the dynamic shared memory limit, raised per device and token count when a
+  // call needs more than the last one did
+  static size_t attr_smem[64][mk::q4::TMAX + 1] = {};
+  if (dev < 0 || dev >= 64) return MK_ERR_UNSUPPORTED;
+  if (attr_smem[dev][T] < smem) {
+    const void* fns[mk::q4::TMAX + 1] = {
+        nullptr,
+        reinterpret_cast<const void*>(mk::q4::gemv_w4_kernel<1>),
+        reinterpret_cast<const void*>(mk::q4::gemv_w4_kernel<2>),
+        reinterpret_cast<const void*>(mk::q4::gemv_w4_kernel<3>),
+        reinterpret_cast<const void*>(mk::q4::gemv_w4_kernel<4>),
+        reinterpret_cast<const void*>(mk::q4::gemv_w4_kernel<5>),
+        reinterpret_cast<const void*>(mk::q4::gemv_w4_kernel<6>),
+        reinterpret_cast<const void*>(mk::q4::gemv_w4_kernel<7>),
+        reinterpret_cast<const void*>(mk::q4::gemv_w4_kernel<8>)};
+    r = cudaFuncSetAttribute(fns[T], cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (r != cudaSuccess) return cuda_status(r);
+    attr_smem[dev][T] = smem;
+  }
+  const int kw = mk::q4::pick_kw(cols);
+  const int rw = mk::q4::rw_for(T);
+  const int rpb = (mk::q4::WARPS / kw) * rw;
+  const int nblk = (rows + rpb - 1) / rpb;
+  const dim3 grid(nblk < mk::q4::MAX_CTAS ? nblk : mk::q4::MAX_CTAS), block(mk::q4::THREADS);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const uint8_t* c = static_cast<const uint8_t*>(codes);
+  switch (T) {
+    case 1: mk::q4::gemv_w4_kernel<1><<<grid, block, smem, st>>>(c, scales, x, rows, cols, y, kw); break;
+    case 2: mk::q4::gemv_w4_kernel<2><<<grid, block, smem, st>>>(c, scales, x, rows, cols, y, kw); break;
+    case 3: mk::q4::gemv_w4_kernel<3><<<grid, block, smem, st>>>(c, scales, x, rows, cols, y, kw); break;
+    case 4: mk::q4::gemv_w4_kernel<4><<<grid, block, smem, st>>>(c, scales, x, rows, cols, y, kw); break;
+    case 5: mk::q4::gemv_w4_kernel<5><<<grid, block, smem, st>>>(c, scales, x, rows, cols, y, kw); break;
+    case 6: mk::q4::gemv_w4_kernel<6><<<grid, block, smem, st>>>(c, scales, x, rows, cols, y, kw); break;
+    case 7: mk::q4::gemv_w4_kernel<7><<<grid, block, smem, st>>>(c, scales, x, rows, cols, y, kw); break;
+    default: mk::q4::gemv_w4_kernel<8><<<grid, block, smem, st>>>(c, scales, x, rows, cols, y, kw); break;
+  }
   return cuda_status(cudaGetLastError());
 }
 

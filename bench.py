@@ -45,11 +45,12 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extras", action="store_true",
                    help="skip the long-context, verify, prefill-roofline and delta-sweep lines")
-    p.add_argument("--mode", choices=["full", "kernel", "delta", "verify"], default="full",
+    p.add_argument("--mode", choices=["full", "kernel", "delta", "verify", "w4"], default="full",
                    help="small cases for profilers: kernel = W+K single decode launches "
                         "at context --ctx on a seeded synthetic state; delta = W+K "
                         "isolated delta steps at batch --batch; verify = W+K 5-token "
-                        "verify calls at context 4096")
+                        "verify calls at context 4096; w4 = the 4-bit weight GEMV at the "
+                        "LM head's shape")
     p.add_argument("--ctx", type=int, default=520, help="context of --mode kernel")
     p.add_argument("--batch", type=int, default=8, help="sequences of --mode delta")
     return p.parse_args()
@@ -403,10 +404,49 @@ def state_to_device(torch, np, st):
                 if isinstance(v, np.ndarray) else v) for k, v in st.items()}
 
 
+def w4_gemv_lines(mk, torch, hbm):
+    """4-bit weight GEMV (mk_gemv_w4) at the tied LM head's shape (151,936 x
+    1024) for 1 and 5 activation rows: three quantised copies used in turn,
+    so each launch reads a matrix the one before did not (3 x 97 MB > the
+    126 MB L2)."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    rows, cols = 151936, 1024
+    g = torch.Generator(device="cuda").manual_seed(12)
+    sets = []
+    for _ in range(3):
+        W = (torch.randn((rows, cols), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device="cuda")
+        scales = torch.empty((rows, cols // 64), dtype=torch.float32, device="cuda")
+        mk.quantize_w4(W.view(torch.int16), codes, scales)
+        sets.append((codes, scales))
+        del W
+    w4 = {}
+    for T in (1, 5):
+        x = torch.randn((T, cols), generator=g, device="cuda")
+        y = torch.empty((T, rows), dtype=torch.float32, device="cuda")
+        for i in range(6):
+            mk.gemv_w4(sets[i % 3][0], sets[i % 3][1], x, y)
+        torch.cuda.synchronize()
+        n = 60
+        e0.record()
+        for i in range(n):
+            mk.gemv_w4(sets[i % 3][0], sets[i % 3][1], x, y)
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1000.0 / n
+        byts = rows * cols // 2 + rows * cols // 64 * 4 + T * cols * 4 + T * rows * 4
+        w4["T%d" % T] = {"us_per_launch": us, "GBps": byts / us / 1e3,
+                         "frac": byts / us / 1e3 / hbm, "bytes_per_launch": byts,
+                         "bf16_equivalent_bytes": rows * cols * 2}
+    del sets
+    return w4
+
+
 def extra_workloads(mk, synth, torch, np, prefill_ms_per_call, hbm, tc_peak, peak_kind):
     """The other configurations of the method, each timed on the device with
     CUDA events: long-context decode, 5-token verify, the prompt path's
-    tensor-core roofline and the isolated delta-step sweep."""
+    tensor-core roofline, the isolated delta-step sweep and the 4-bit weight
+    GEMV."""
     out = {}
     # prompt path: algorithmic FLOPs of pp520 (every matrix once per position,
     # LM head for the last position only) over the measured prefill time
@@ -537,6 +577,8 @@ def extra_workloads(mk, synth, torch, np, prefill_ms_per_call, hbm, tc_peak, pea
                             "launch": "CUDA graph of %d launches" % steps}
         del S, q, k, q16, k16, v16, be, al, o
     out["delta_sweep_dk128_h16"] = sweep
+
+    out["gemv_w4_lmhead_151936x1024"] = w4_gemv_lines(mk, torch, hbm)
     return out
 
 
@@ -553,6 +595,15 @@ def main():
         return
     if args.mode == "verify":
         run_verify_mode(args)
+        return
+    if args.mode == "w4":
+        import torch
+        import attention_decode_megakernel_b200 as mk
+        from attention_decode_megakernel_b200 import build
+        build.build()
+        hbm, _, _ = peaks()
+        print(json.dumps({"mode": "w4", "gemv_w4_lmhead_151936x1024":
+                          w4_gemv_lines(mk, torch, hbm)}), flush=True)
         return
     if args.mode == "kernel":
         run_kernel_mode(args)

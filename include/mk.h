@@ -325,6 +325,39 @@ int mk_debug_gemm(const void *W, const void *X, float *C, int n_out, int T,
 int mk_debug_gemm_noalloc(const void *W, const void *X, float *C, int n_out,
                           int T, int K, void *stream);
 
+/* ---- 4-bit weights ------------------------------------------------------
+ * The tag page "RTX 3090" (item on a custom engine for a 27B-class model
+ * on one RTX 3090: 4-bit weights with 16-bit activations, "W4A16") credits
+ * 4-bit weights for its speed, since a batch-1 decoder streams every weight
+ * once per token.  Format (the page names none; this is the plain
+ * group-wise symmetric reading): groups of 64 consecutive weights of a row
+ * share one fp32 scale s = max|w| / 7 (0 for an all-zero group); each weight
+ * is stored as the nibble q + 8 with q = clamp(rint(w / s), -7, 7) (IEEE
+ * fp32 division, round half to even); weight k of a row lives in byte k / 2
+ * of the row, the even weight in the low nibble.  A row of `cols` weights
+ * takes cols / 2 bytes of codes and cols / 16 bytes of scales. */
+
+/* Quantise W (device, bf16 [rows][cols], 16-byte aligned) into codes
+ * (device, uint8 [rows][cols / 2], 16-byte aligned) and scales (device,
+ * float32 [rows][cols / 64], 16-byte aligned).  cols must be a multiple of
+ * 64 (else MK_ERR_ARG).  Asynchronous on `stream` (a cudaStream_t or NULL);
+ * nothing is allocated. */
+int mk_quantize_w4(const void *W, int rows, int cols, void *codes, float *scales,
+                   void *stream);
+
+/* y[t][n] = sum_k s(n, k / 64) * q(n, k) * x[t][k] for t < T, with fp32
+ * activations and fp32 accumulation: every code row is read once for all T
+ * rows of x.  codes / scales as mk_quantize_w4 writes them; x (device,
+ * float32 [T][cols], 16-byte aligned); y (device, float32 [T][rows]).
+ * 1 <= T <= 8 and cols a multiple of 64 (else MK_ERR_ARG); T * cols * 4
+ * bytes must fit in 220 KB of shared memory (else MK_ERR_UNSUPPORTED).
+ * Asynchronous on `stream`; allocates nothing.  The first call per device
+ * and T (and any call that needs more shared memory than the earlier ones)
+ * raises the kernel's shared-memory limit: serialise those calls when
+ * several host threads use the library. */
+int mk_gemv_w4(const void *codes, const float *scales, const float *x, int T,
+               int rows, int cols, float *y, void *stream);
+
 /* Human-readable text of a status code. */
 const char *mk_strerror(int status);
 

@@ -69,6 +69,9 @@ def lib():
             getattr(L, f).restype = C.c_double
             getattr(L, f).argtypes = [C.c_double]
         L.orc_gemv.argtypes = [C.c_void_p, C.c_int, C.c_int, _D, _D]
+        L.orc_quantize_w4.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]
+        L.orc_dequantize_w4.argtypes = [C.c_void_p, C.c_void_p, C.c_int, C.c_int, _D]
+        L.orc_gemv_w4.argtypes = [C.c_void_p, C.c_void_p, C.c_int, C.c_int, _D, _D]
         L.orc_set_threads.argtypes = [C.c_int]
         L.orc_set_threads.restype = None
         L.orc_rmsnorm.argtypes = [_D, C.c_void_p, C.c_int, C.c_double, _D]
@@ -131,6 +134,38 @@ def gemv(W_bits: np.ndarray, x: np.ndarray) -> np.ndarray:
     x = np.ascontiguousarray(x, dtype=np.float64)
     y = np.zeros(W_bits.shape[0], np.float64)
     lib().orc_gemv(_vp(W_bits), W_bits.shape[0], W_bits.shape[1], _dp(x), _dp(y))
+    return y
+
+
+def quantize_w4(W_bits: np.ndarray):
+    """4-bit group-wise codes (uint8 [rows][cols/2]) and scales (float32
+    [rows][cols/64]) of a bf16 matrix given as uint16 bits."""
+    W_bits = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    rows, cols = W_bits.shape
+    if cols % 64:
+        raise ValueError("cols must be a multiple of 64")
+    codes = np.zeros((rows, cols // 2), dtype=np.uint8)
+    scales = np.zeros((rows, cols // 64), dtype=np.float32)
+    lib().orc_quantize_w4(_vp(W_bits), rows, cols, _vp(codes), _vp(scales))
+    return codes, scales
+
+
+def dequantize_w4(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    rows, half = codes.shape
+    Wd = np.zeros((rows, 2 * half), dtype=np.float64)
+    lib().orc_dequantize_w4(_vp(codes), _vp(scales), rows, 2 * half, _dp(Wd))
+    return Wd
+
+
+def gemv_w4(codes: np.ndarray, scales: np.ndarray, x: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    rows, half = codes.shape
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    y = np.zeros(rows, dtype=np.float64)
+    lib().orc_gemv_w4(_vp(codes), _vp(scales), rows, 2 * half, _dp(x), _dp(y))
     return y
 
 

@@ -94,6 +94,66 @@ void orc_gemv(const uint16_t *W, int rows, int cols, const double *x, double *y)
   }
 }
 
+/* 4-bit weights (tag page "RTX 3090", item on a custom engine for a
+ * 27B-class model: 4-bit weights with 16-bit activations).  The page names
+ * no format; the reading taken: groups of 64 consecutive weights of a row
+ * share the scale s = max|w| / 7, each weight becomes q = clamp(rint(w / s),
+ * -7, 7) stored as the nibble q + 8, weight k in byte k / 2 (even k in the
+ * low nibble).  The scale and the code are decided in fp32 (IEEE division,
+ * round half to even), the precision the kernel decides them in; the
+ * dequantised weight q * s and everything after it are double. */
+void orc_quantize_w4(const uint16_t *W, int rows, int cols, uint8_t *codes, float *scales) {
+  const int gpr = cols / 64;
+  for (int r = 0; r < rows; ++r)
+    for (int g = 0; g < gpr; ++g) {
+      const uint16_t *w = W + (long)r * cols + g * 64;
+      float amax = 0.0f;
+      for (int k = 0; k < 64; ++k) {
+        const float v = fabsf((float)bfw(w, k));
+        if (v > amax) amax = v;
+      }
+      const float s = amax / 7.0f;
+      scales[(long)r * gpr + g] = s;
+      uint8_t *c = codes + (long)r * (cols / 2) + g * 32;
+      for (int k = 0; k < 64; k += 2) {
+        int q[2] = {0, 0};
+        for (int e = 0; e < 2; ++e) {
+          if (s > 0.0f) {
+            const float ratio = (float)bfw(w, k + e) / s;
+            int v = (int)nearbyintf(ratio);
+            q[e] = v < -7 ? -7 : v > 7 ? 7 : v;
+          }
+        }
+        c[k / 2] = (uint8_t)((q[0] + 8) | ((q[1] + 8) << 4));
+      }
+    }
+}
+
+/* Wd[r][k] = (nibble(r, k) - 8) * s(r, k / 64), in double. */
+void orc_dequantize_w4(const uint8_t *codes, const float *scales, int rows, int cols,
+                       double *Wd) {
+  for (int r = 0; r < rows; ++r)
+    for (int k = 0; k < cols; ++k) {
+      const uint8_t b = codes[(long)r * (cols / 2) + k / 2];
+      const int nibble = (k % 2 == 0) ? (b & 0xF) : (b >> 4);
+      Wd[(long)r * cols + k] = (double)(nibble - 8) * (double)scales[(long)r * (cols / 64) + k / 64];
+    }
+}
+
+/* y = Wd x with the dequantised weights, one row at a time. */
+void orc_gemv_w4(const uint8_t *codes, const float *scales, int rows, int cols, const double *x,
+                 double *y) {
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < rows; ++r) {
+    double *wd = (double *)malloc(sizeof(double) * cols);
+    orc_dequantize_w4(codes + (long)r * (cols / 2), scales + (long)r * (cols / 64), 1, cols, wd);
+    double acc = 0.0;
+    for (int k = 0; k < cols; ++k) acc += wd[k] * x[k];
+    y[r] = acc;
+    free(wd);
+  }
+}
+
 /* RMSNorm: y = x / sqrt(mean(x^2) + eps) * w  (w == NULL means gain 1). */
 void orc_rmsnorm(const double *x, const uint16_t *w, int n, double eps, double *y) {
   double ss = 0.0;

@@ -55,6 +55,11 @@ double orc_sigmoid(double x);
 double orc_softplus(double x);
 double orc_silu(double x);
 void orc_gemv(const uint16_t *W, int rows, int cols, const double *x, double *y);
+void orc_quantize_w4(const uint16_t *W, int rows, int cols, uint8_t *codes, float *scales);
+void orc_dequantize_w4(const uint8_t *codes, const float *scales, int rows, int cols,
+                       double *Wd);
+void orc_gemv_w4(const uint8_t *codes, const float *scales, int rows, int cols, const double *x,
+                 double *y);
 void orc_rmsnorm(const double *x, const uint16_t *w, int n, double eps, double *y);
 void orc_l2norm(const double *x, int n, double eps, double *y);
 void orc_causal_conv_step(int channels, int K, const uint16_t *w, double *state,
