@@ -1,6 +1,7 @@
 // mk_engine.cu -- host side of the C ABI declared in include/mk.h: config
 // validation, workspace carve-up, cooperative launches of the decode kernel,
-// state rotation for verify checkpoints, state I/O and error reporting.
+// state buffer rotation, verify records and their replay, state I/O and error
+// reporting.
 #include <cuda_runtime.h>
 
 #include <cstdio>

@@ -40,7 +40,8 @@ struct DevModel {
   // weights
   const uint16_t *embed, *final_norm;
   DevLayer layers[MK_MAX_LAYERS];
-  // recurrent state: kStateBufs rotating buffers (current + verify checkpoints)
+  // recurrent state: kStateBufs rotating buffers (current, next, and the
+  // per-position copies of the decode-launch verify fallback)
   float *dn_state[kStateBufs];      // [n_dn][nh][dv][dk]
   float *conv_state[kStateBufs];    // [n_dn][ch][4]  (3 taps of history + pad)
   uint16_t *kc, *vc;                // [n_attn][nkv][max_ctx][hd]
