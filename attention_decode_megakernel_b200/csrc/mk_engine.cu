@@ -400,6 +400,29 @@ int launch_pdl(mk_engine* e, void (*kern)(KArgs...), dim3 grid, dim3 block, size
   return cuda_status(r);
 }
 
+// The chunk attention instantiation for qt (the query rows rounded up to 8).
+template <int HD>
+int launch_attn_chunk(mk_engine* e, int qt, dim3 grid, dim3 block, const mk::vf::AttArgs& aa) {
+  switch (qt) {
+    case 8: return launch_pdl(e, mk::vf::attn_chunk_kernel<HD, 8>, grid, block, mk::vf::att_smem<HD, 8>(), aa);
+    case 16: return launch_pdl(e, mk::vf::attn_chunk_kernel<HD, 16>, grid, block, mk::vf::att_smem<HD, 16>(), aa);
+    case 24: return launch_pdl(e, mk::vf::attn_chunk_kernel<HD, 24>, grid, block, mk::vf::att_smem<HD, 24>(), aa);
+    default: return launch_pdl(e, mk::vf::attn_chunk_kernel<HD, 32>, grid, block, mk::vf::att_smem<HD, 32>(), aa);
+  }
+}
+
+template <int HD>
+bool attn_chunk_attrs() {
+  return cudaFuncSetAttribute(mk::vf::attn_chunk_kernel<HD, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              int(mk::vf::att_smem<HD, 8>())) == cudaSuccess &&
+         cudaFuncSetAttribute(mk::vf::attn_chunk_kernel<HD, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              int(mk::vf::att_smem<HD, 16>())) == cudaSuccess &&
+         cudaFuncSetAttribute(mk::vf::attn_chunk_kernel<HD, 24>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              int(mk::vf::att_smem<HD, 24>())) == cudaSuccess &&
+         cudaFuncSetAttribute(mk::vf::attn_chunk_kernel<HD, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              int(mk::vf::att_smem<HD, 32>())) == cudaSuccess;
+}
+
 // One skinny projection (a chunk of T <= 8 tokens): grid of at most two
 // CTAs per SM over the output's row blocks, launched so that it may start
 // (and stream its first weights) while the kernel before it finishes.
@@ -690,13 +713,14 @@ int run_chunk(mk_engine* e, const int32_t* tokens_host, int T, const VerifyPlan*
         aa.out = Af;
         aa.ldo = aw;
         const dim3 ag(aa.nsplit, nkv), mg(nq, T), tb(mk::vf::ATT_THREADS);
+        const int qt = ((nq / nkv) * T + 7) / 8 * 8;
         if (rc == MK_OK) {
           if (hd == 256)
-            rc = launch_pdl(e, mk::vf::attn_chunk_kernel<256>, ag, tb, mk::vf::att_smem<256>(), aa);
+            rc = launch_attn_chunk<256>(e, qt, ag, tb, aa);
           else if (hd == 128)
-            rc = launch_pdl(e, mk::vf::attn_chunk_kernel<128>, ag, tb, mk::vf::att_smem<128>(), aa);
+            rc = launch_attn_chunk<128>(e, qt, ag, tb, aa);
           else
-            rc = launch_pdl(e, mk::vf::attn_chunk_kernel<64>, ag, tb, mk::vf::att_smem<64>(), aa);
+            rc = launch_attn_chunk<64>(e, qt, ag, tb, aa);
         }
         if (rc == MK_OK) {
           if (hd == 256)
@@ -1096,15 +1120,7 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
                         (c.dn_heads * c.dn_dv) % 4 == 0 && e->hm.ch % 4 == 0 && c.mlp % 8 == 0 &&
                         (c.q_heads * c.head_dim) % 8 == 0;
     e->sk_ok = smem <= 227u * 1024u && c.dn_dv % 32 == 0 && rows16 && skinny_attrs(smem) &&
-               cudaFuncSetAttribute(mk::vf::attn_chunk_kernel<256>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    int(mk::vf::att_smem<256>())) == cudaSuccess &&
-               cudaFuncSetAttribute(mk::vf::attn_chunk_kernel<128>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    int(mk::vf::att_smem<128>())) == cudaSuccess &&
-               cudaFuncSetAttribute(mk::vf::attn_chunk_kernel<64>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    int(mk::vf::att_smem<64>())) == cudaSuccess;
+               attn_chunk_attrs<256>() && attn_chunk_attrs<128>() && attn_chunk_attrs<64>();
   }
   cudaGetLastError();
   {

@@ -302,10 +302,12 @@ constexpr int ATT_L = 32;      // keys per range (two CTAs per SM over 4K keys)
 constexpr int ATT_QMAX = 32;   // query rows per kv head (G * T)
 constexpr int ATT_THREADS = 256;
 
-template <int HD>
+// QT: the query rows G * T rounded up to a multiple of 8 (one instantiation
+// each, so the loops carry no idle rows beyond the last group of 8)
+template <int HD, int QT>
 constexpr size_t att_smem() {
-  return size_t(ATT_L) * (HD + 8) * 2 + size_t(ATT_L) * HD * 2 + size_t(ATT_QMAX) * HD * 4 +
-         size_t(ATT_QMAX) * ATT_L * 4;
+  return size_t(ATT_L) * (HD + 8) * 2 + size_t(ATT_L) * HD * 2 + size_t(QT) * HD * 4 +
+         size_t(QT) * ATT_L * 4;
 }
 
 struct AttArgs {
@@ -319,15 +321,15 @@ struct AttArgs {
   int ldo;
 };
 
-template <int HD>
+template <int HD, int QT>
 __global__ void __launch_bounds__(ATT_THREADS, 2) attn_chunk_kernel(const __grid_constant__ AttArgs a) {
   extern __shared__ __align__(16) unsigned char att_sm[];
   constexpr int KLD = HD + 8;  // padded key row: conflict-free 16-byte row reads
   uint16_t* Ks = reinterpret_cast<uint16_t*>(att_sm);     // [L][KLD]
   uint16_t* Vs = Ks + ATT_L * KLD;                        // [L][HD]
-  float* Qs = reinterpret_cast<float*>(Vs + ATT_L * HD);  // [QMAX][HD], scaled by HD^-1/2
-  float* Ps = Qs + ATT_QMAX * HD;                         // [QMAX][L] scores, then weights
-  __shared__ float ms[ATT_QMAX], ls[ATT_QMAX];
+  float* Qs = reinterpret_cast<float*>(Vs + ATT_L * HD);  // [QT][HD], scaled by HD^-1/2
+  float* Ps = Qs + QT * HD;                               // [QT][L] scores, then weights
+  __shared__ float ms[QT], ls[QT];
   griddep_launch_dependents();
   const int s = blockIdx.x, g = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = a.nq / a.nkv, Q = G * a.T;
@@ -360,11 +362,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_chunk_kernel(const __grid
   __syncthreads();
   // ---- scores: thread (key j, query group qg), queries qg + SQG r ---------------
   {
-    constexpr int SQG = ATT_THREADS / ATT_L, SQPT = ATT_QMAX / SQG;
+    constexpr int SQG = ATT_THREADS / ATT_L, SQPT = QT / SQG;
     const int j = tid % ATT_L, qg = tid / ATT_L, kp = k0 + j;
-    float sc[SQPT];
+    float sa[SQPT], sb[SQPT];  // even / odd dimensions (packed FMAs)
 #pragma unroll
-    for (int r = 0; r < SQPT; ++r) sc[r] = 0.f;
+    for (int r = 0; r < SQPT; ++r) sa[r] = sb[r] = 0.f;
     const uint16_t* kr = Ks + j * KLD;
     for (int d = 0; d < HD; d += 8) {
       const uint4 u = *reinterpret_cast<const uint4*>(kr + d);
@@ -376,16 +378,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_chunk_kernel(const __grid
         if (qi < Q) {
           const float4 q0 = *reinterpret_cast<const float4*>(Qs + qi * HD + d);
           const float4 q1 = *reinterpret_cast<const float4*>(Qs + qi * HD + d + 4);
-          float acc = sc[r];
-          acc = fmaf(q0.x, kf[0], acc);
-          acc = fmaf(q0.y, kf[1], acc);
-          acc = fmaf(q0.z, kf[2], acc);
-          acc = fmaf(q0.w, kf[3], acc);
-          acc = fmaf(q1.x, kf[4], acc);
-          acc = fmaf(q1.y, kf[5], acc);
-          acc = fmaf(q1.z, kf[6], acc);
-          acc = fmaf(q1.w, kf[7], acc);
-          sc[r] = acc;
+          ffma2(sa[r], sb[r], q0.x, q0.y, kf[0], kf[1]);
+          ffma2(sa[r], sb[r], q0.z, q0.w, kf[2], kf[3]);
+          ffma2(sa[r], sb[r], q1.x, q1.y, kf[4], kf[5]);
+          ffma2(sa[r], sb[r], q1.z, q1.w, kf[6], kf[7]);
         }
       }
     }
@@ -394,7 +390,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_chunk_kernel(const __grid
       const int qi = qg + SQG * r;
       if (qi < Q) {
         const int t = qi / G;  // causal: key position <= the query's position
-        Ps[qi * ATT_L + j] = (kp < k1 && kp <= a.pos0 + t) ? sc[r] : -INFINITY;
+        Ps[qi * ATT_L + j] = (kp < k1 && kp <= a.pos0 + t) ? sa[r] + sb[r] : -INFINITY;
       }
     }
   }
@@ -425,7 +421,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_chunk_kernel(const __grid
   __syncthreads();
   // ---- weighted values: thread (4 dims, query group), queries qg + PQG r -------
   {
-    constexpr int DG = HD / 4, PQG = ATT_THREADS / DG, PQPT = ATT_QMAX / PQG;
+    constexpr int DG = HD / 4, PQG = ATT_THREADS / DG, PQPT = (QT + PQG - 1) / PQG;
     const int dg = tid % DG, qg = tid / DG, nk = k1 - k0;
     float acc[PQPT][4];
 #pragma unroll
@@ -438,10 +434,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_chunk_kernel(const __grid
         const int qi = qg + PQG * r;
         if (qi < Q) {
           const float p = Ps[qi * ATT_L + j];
-          acc[r][0] = fmaf(p, v0, acc[r][0]);
-          acc[r][1] = fmaf(p, v1, acc[r][1]);
-          acc[r][2] = fmaf(p, v2, acc[r][2]);
-          acc[r][3] = fmaf(p, v3, acc[r][3]);
+          ffma2(acc[r][0], acc[r][1], p, p, v0, v1);
+          ffma2(acc[r][2], acc[r][3], p, p, v2, v3);
         }
       }
     }
