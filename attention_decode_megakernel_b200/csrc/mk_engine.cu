@@ -762,7 +762,29 @@ int run_chunk(mk_engine* e, const int32_t* tokens_host, int T, const VerifyPlan*
                                                              c.rope_theta);
         e->launches += 2;  // rope, attention
         const dim3 agrid((T + 7) / 8, nq);
-        if (hd == 256)
+        mk::vf::PromptAttArgs pa{};
+        pa.P = P;
+        pa.ldp = pw;
+        pa.kc = m.kc + kvo;
+        pa.vc = m.vc + kvo;
+        pa.max_ctx = c.max_ctx;
+        pa.nq = nq;
+        pa.nkv = nkv;
+        pa.pos0 = pos0;
+        pa.T = T;
+        pa.Ob = A16;
+        pa.ldo = aw;
+        pa.lo = lo_a;
+        const dim3 pg((T + mk::vf::PR_POS - 1) / mk::vf::PR_POS, nkv), pb(mk::vf::ATT_THREADS);
+        // flash-style tiles when a block's query rows fit one CTA
+        const bool flash = e->sk_ok && (nq / nkv) * mk::vf::PR_POS <= mk::vf::ATT_QMAX;
+        if (flash && hd == 256)
+          mk::vf::attn_prompt_kernel<256><<<pg, pb, mk::vf::prompt_att_smem<256>(), st>>>(pa);
+        else if (flash && hd == 128)
+          mk::vf::attn_prompt_kernel<128><<<pg, pb, mk::vf::prompt_att_smem<128>(), st>>>(pa);
+        else if (flash)
+          mk::vf::attn_prompt_kernel<64><<<pg, pb, mk::vf::prompt_att_smem<64>(), st>>>(pa);
+        else if (hd == 256)
           attn_prefill_kernel<256><<<agrid, 256, 0, st>>>(P, pw, m.kc + kvo, m.vc + kvo,
                                                           c.max_ctx, nq, nkv, pos0, T, A16, aw,
                                                           lo_a);
@@ -1120,7 +1142,16 @@ int mk_create(const mk_config* cfg, const mk_weights* w, void* workspace, size_t
                         (c.dn_heads * c.dn_dv) % 4 == 0 && e->hm.ch % 4 == 0 && c.mlp % 8 == 0 &&
                         (c.q_heads * c.head_dim) % 8 == 0;
     e->sk_ok = smem <= 227u * 1024u && c.dn_dv % 32 == 0 && rows16 && skinny_attrs(smem) &&
-               attn_chunk_attrs<256>() && attn_chunk_attrs<128>() && attn_chunk_attrs<64>();
+               attn_chunk_attrs<256>() && attn_chunk_attrs<128>() && attn_chunk_attrs<64>() &&
+               cudaFuncSetAttribute(mk::vf::attn_prompt_kernel<256>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    int(mk::vf::prompt_att_smem<256>())) == cudaSuccess &&
+               cudaFuncSetAttribute(mk::vf::attn_prompt_kernel<128>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    int(mk::vf::prompt_att_smem<128>())) == cudaSuccess &&
+               cudaFuncSetAttribute(mk::vf::attn_prompt_kernel<64>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    int(mk::vf::prompt_att_smem<64>())) == cudaSuccess;
   }
   cudaGetLastError();
   {

@@ -29,6 +29,7 @@
 #include <cooperative_groups.h>
 
 #include "mk_model.cuh"
+#include "mk_prefill.cuh"
 #include "mk_ptx.cuh"
 
 namespace mk {
@@ -522,6 +523,180 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_chunk_merge(const __grid_con
         den = fmaf(c, wl[w], den);
       }
     a.out[size_t(t) * a.ldo + h * HD + d] = num / den;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Causal GQA attention of a prompt chunk, flash style: one CTA per (block of
+// 8 positions, kv head) holds the block's G x 8 query rows and walks the key
+// positions 0 .. its last position in tiles of 32 (K and V double-buffered
+// with cp.async), keeping a running max, sum and weighted value sum per row
+// (online softmax), so no partials leave the CTA.  Scores and the weighted
+// sum use the chunk kernel's thread layout and packed FMAs.  The output
+// rows go out as split bf16 operands (hi, lo) of the output projection GEMM.
+constexpr int PR_POS = 8;  // positions per CTA (x G query rows <= 32)
+
+template <int HD>
+constexpr size_t prompt_att_smem() {
+  return size_t(2) * ATT_L * (HD + 8) * 2 + size_t(2) * ATT_L * HD * 2 +
+         size_t(ATT_QMAX) * HD * 4 + size_t(ATT_QMAX) * ATT_L * 4;
+}
+
+struct PromptAttArgs {
+  const float* P;      // [T][ldp] rotated q of head h at column h * HD
+  int ldp;
+  const uint16_t* kc;  // [nkv][max_ctx][HD] bf16, positions < pos0 + T written
+  const uint16_t* vc;
+  int max_ctx, nq, nkv, pos0, T;
+  uint16_t* Ob;        // [T][ldo] bf16 hi (+ lo at offset lo), head h at column h * HD
+  int ldo;
+  size_t lo;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(ATT_THREADS, 2) attn_prompt_kernel(
+    const __grid_constant__ PromptAttArgs a) {
+  extern __shared__ __align__(16) unsigned char pa_sm[];
+  constexpr int KLD = HD + 8, L = ATT_L;
+  uint16_t* Ks = reinterpret_cast<uint16_t*>(pa_sm);       // [2][L][KLD]
+  uint16_t* Vs = Ks + 2 * L * KLD;                         // [2][L][HD]
+  float* Qs = reinterpret_cast<float*>(Vs + 2 * L * HD);   // [32][HD], scaled by HD^-1/2
+  float* Ps = Qs + ATT_QMAX * HD;                          // [32][L]
+  __shared__ float mrow[ATT_QMAX], lrow[ATT_QMAX], crow[ATT_QMAX];
+  const int b = blockIdx.x, g = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.nq / a.nkv;
+  const int t0 = b * PR_POS, tb = min(PR_POS, a.T - t0), R = tb * G;
+  const int kend = a.pos0 + t0 + tb;  // keys 0 .. kend - 1 (the block's last position)
+  const int ntile = (kend + L - 1) / L;
+  const uint16_t* K = a.kc + size_t(g) * a.max_ctx * HD;
+  const uint16_t* V = a.vc + size_t(g) * a.max_ctx * HD;
+  constexpr int VPR = HD / 8;
+  auto stage = [&](int tile) {
+    const int j0 = tile * L, j1 = min(j0 + L, kend), buf = tile & 1;
+    for (int i = tid; i < (j1 - j0) * VPR; i += ATT_THREADS) {
+      const int j = i / VPR, c = i % VPR;
+      cp_async16(Ks + (buf * L + j) * KLD + c * 8, K + size_t(j0 + j) * HD + c * 8);
+      cp_async16(Vs + (buf * L + j) * HD + c * 8, V + size_t(j0 + j) * HD + c * 8);
+    }
+  };
+  stage(0);
+  cp_async_commit();
+  const float scale = 1.0f / sqrtf(float(HD));
+  for (int i = tid; i < R * (HD / 4); i += ATT_THREADS) {
+    const int r = i / (HD / 4), c = i % (HD / 4);
+    const int t = r / G, gi = r - t * G;
+    float4 q = *reinterpret_cast<const float4*>(a.P + size_t(t0 + t) * a.ldp + (g * G + gi) * HD +
+                                                c * 4);
+    q.x *= scale;
+    q.y *= scale;
+    q.z *= scale;
+    q.w *= scale;
+    *reinterpret_cast<float4*>(Qs + r * HD + c * 4) = q;
+  }
+  if (tid < ATT_QMAX) {
+    mrow[tid] = -INFINITY;
+    lrow[tid] = 0.f;
+  }
+  constexpr int DG = HD / 4, PQG = ATT_THREADS / DG, PQPT = (ATT_QMAX + PQG - 1) / PQG;
+  const int dg = tid % DG, pqg = tid / DG;
+  float acc[PQPT][4];
+#pragma unroll
+  for (int r = 0; r < PQPT; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+  constexpr int SQG = ATT_THREADS / L, SQPT = ATT_QMAX / SQG;
+  const int j = tid % L, sqg = tid / L;
+  for (int tile = 0; tile < ntile; ++tile) {
+    if (tile + 1 < ntile) stage(tile + 1);
+    cp_async_commit();
+    cp_async_wait_all_but_one();  // this tile's keys and values have landed
+    __syncthreads();
+    const int buf = tile & 1, k0 = tile * L, nk = min(L, kend - k0);
+    // scores of the tile, masked by position
+    {
+      float sa[SQPT], sb[SQPT];
+#pragma unroll
+      for (int r = 0; r < SQPT; ++r) sa[r] = sb[r] = 0.f;
+      const uint16_t* kr = Ks + (buf * L + j) * KLD;
+      for (int d = 0; d < HD; d += 8) {
+        const uint4 u = *reinterpret_cast<const uint4*>(kr + d);
+        const float kf[8] = {bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y),
+                             bf_lo(u.z), bf_hi(u.z), bf_lo(u.w), bf_hi(u.w)};
+#pragma unroll
+        for (int r = 0; r < SQPT; ++r) {
+          const int qi = sqg + SQG * r;
+          if (qi < R) {
+            const float4 q0 = *reinterpret_cast<const float4*>(Qs + qi * HD + d);
+            const float4 q1 = *reinterpret_cast<const float4*>(Qs + qi * HD + d + 4);
+            ffma2(sa[r], sb[r], q0.x, q0.y, kf[0], kf[1]);
+            ffma2(sa[r], sb[r], q0.z, q0.w, kf[2], kf[3]);
+            ffma2(sa[r], sb[r], q1.x, q1.y, kf[4], kf[5]);
+            ffma2(sa[r], sb[r], q1.z, q1.w, kf[6], kf[7]);
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < SQPT; ++r) {
+        const int qi = sqg + SQG * r;
+        if (qi < R) {
+          const int kp = k0 + j, qpos = a.pos0 + t0 + qi / G;
+          Ps[qi * L + j] = (j < nk && kp <= qpos) ? sa[r] + sb[r] : -INFINITY;
+        }
+      }
+    }
+    __syncthreads();
+    // online softmax: one warp per row, one key per lane (L == 32)
+    for (int qi = warp; qi < R; qi += ATT_THREADS / 32) {
+      const float s = Ps[qi * L + lane];
+      const float mo = mrow[qi], mn = fmaxf(mo, warp_max(s));
+      const float p = mn == -INFINITY ? 0.f : expf(s - mn);
+      const float c = mo == -INFINITY ? 0.f : expf(mo - mn);
+      const float ps = warp_sum(p);
+      Ps[qi * L + lane] = p;
+      if (lane == 0) {
+        mrow[qi] = mn;
+        lrow[qi] = lrow[qi] * c + ps;
+        crow[qi] = c;
+      }
+    }
+    __syncthreads();
+    // weighted values: rescale the running sums, add the tile
+#pragma unroll
+    for (int r = 0; r < PQPT; ++r) {
+      const int qi = pqg + PQG * r;
+      if (qi < R) {
+        const float c = crow[qi];
+        acc[r][0] *= c;
+        acc[r][1] *= c;
+        acc[r][2] *= c;
+        acc[r][3] *= c;
+      }
+    }
+    for (int jj = 0; jj < nk; ++jj) {
+      const uint2 u = *reinterpret_cast<const uint2*>(Vs + (buf * L + jj) * HD + dg * 4);
+      const float v0 = bf_lo(u.x), v1 = bf_hi(u.x), v2 = bf_lo(u.y), v3 = bf_hi(u.y);
+#pragma unroll
+      for (int r = 0; r < PQPT; ++r) {
+        const int qi = pqg + PQG * r;
+        if (qi < R) {
+          const float p = Ps[qi * L + jj];
+          ffma2(acc[r][0], acc[r][1], p, p, v0, v1);
+          ffma2(acc[r][2], acc[r][3], p, p, v2, v3);
+        }
+      }
+    }
+    __syncthreads();  // the buffers and Ps are reused by the next tile
+  }
+#pragma unroll
+  for (int r = 0; r < PQPT; ++r) {
+    const int qi = pqg + PQG * r;
+    if (qi < R) {
+      const float inv = 1.0f / lrow[qi];
+      const int t = qi / G, h = g * G + (qi - (qi / G) * G);
+      uint16_t* o = a.Ob + size_t(t0 + t) * a.ldo + h * HD + dg * 4;
+      pf::store_split(o + 0, a.lo, acc[r][0] * inv);
+      pf::store_split(o + 1, a.lo, acc[r][1] * inv);
+      pf::store_split(o + 2, a.lo, acc[r][2] * inv);
+      pf::store_split(o + 3, a.lo, acc[r][3] * inv);
+    }
   }
 }
 
