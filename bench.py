@@ -181,24 +181,48 @@ def sustained_tc_peak():
         return FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback sustained"
 
 
-def decode_bytes(cfg, ctx):
-    """Algorithmic HBM bytes of one decode launch at context `ctx` (the new
-    token is position ctx): every weight once (tied embedding read as the LM
-    head), DeltaNet state read+write, conv history read+write, KV read of
-    ctx positions + write of one, logits written."""
+def weight_bytes(cfg):
+    """Every weight once: the layers' tensors, the tied embedding (read as the
+    LM head) and the final norm gain."""
     import numpy as np
     from attention_decode_megakernel_b200 import synth
     n = 0
     for is_attn in cfg.layer_is_attn:
         for _, shape, kind in synth.layer_tensor_shapes(cfg, is_attn):
             n += int(np.prod(shape)) * (4 if kind == "f" else 2)
-    n += cfg.vocab * cfg.hidden * 2 + cfg.hidden * 2
-    n += 2 * cfg.n_dn * cfg.dn_heads * cfg.dn_dv * cfg.dn_dk * 4
-    n += 2 * cfg.n_dn * cfg.conv_channels * (cfg.conv_k - 1) * 4
-    kv_pos = cfg.n_attn * 2 * cfg.kv_heads * cfg.head_dim * 2
-    n += kv_pos * (ctx + 1)
-    n += cfg.vocab * 4
-    return n
+    return n + cfg.vocab * cfg.hidden * 2 + cfg.hidden * 2
+
+
+def state_bytes(cfg):
+    """One read (or one write) of the DeltaNet state and the conv history."""
+    return (cfg.n_dn * cfg.dn_heads * cfg.dn_dv * cfg.dn_dk * 4
+            + cfg.n_dn * cfg.conv_channels * (cfg.conv_k - 1) * 4)
+
+
+def kv_position_bytes(cfg):
+    """K and V of one position in every attention layer (bf16)."""
+    return cfg.n_attn * 2 * cfg.kv_heads * cfg.head_dim * 2
+
+
+def decode_bytes(cfg, ctx):
+    """Algorithmic HBM bytes of one decode launch at context `ctx` (the new
+    token is position ctx): every weight once (tied embedding read as the LM
+    head), DeltaNet state and conv history read + written, KV read of ctx
+    positions + write of one, logits written."""
+    return (weight_bytes(cfg) + 2 * state_bytes(cfg) + kv_position_bytes(cfg) * (ctx + 1)
+            + cfg.vocab * 4)
+
+
+def verify_bytes(cfg, ctx, n, replayed):
+    """Algorithmic HBM bytes of one n-token verify call at context ctx whose
+    previous accept kept `replayed` positions: every weight once; the state
+    read once and, replayed, written once to the next buffer; n records
+    written (per DeltaNet layer and position: key, value, alpha, beta and
+    the conv inputs) and the replayed ones read; KV read over the context
+    and n positions appended; n rows of logits."""
+    rec = cfg.n_dn * (cfg.dn_heads * (cfg.dn_dk + cfg.dn_dv + 2) + cfg.conv_channels) * 4
+    return (weight_bytes(cfg) + 2 * state_bytes(cfg) + (n + replayed) * rec
+            + kv_position_bytes(cfg) * (ctx + n) + n * cfg.vocab * 4)
 
 
 class Clocks:
@@ -517,19 +541,8 @@ def extra_workloads(mk, synth, torch, np, prefill_ms_per_call, hbm, tc_peak, pea
     eng.sync()
     wall = time.perf_counter() - t0
     dev_ms = e0.elapsed_time(e1)
-    weights = decode_bytes(cfg, 0) - cfg.vocab * 4 - 2 * cfg.n_attn * 2 * cfg.kv_heads * cfg.head_dim * 2
-    dn = cfg.n_dn * cfg.dn_heads * cfg.dn_dv * cfg.dn_dk * 4
-    conv = cfg.n_dn * cfg.conv_channels * (cfg.conv_k - 1) * 4
-    kvb = cfg.n_attn * 2 * cfg.kv_heads * cfg.head_dim * 2
-    # per DeltaNet layer and position: key, value, alpha, beta, conv inputs
-    rec = cfg.n_dn * (cfg.dn_heads * (cfg.dn_dk + cfg.dn_dv + 2) + cfg.conv_channels) * 4
-    acc = kept / calls
-    # weights once; the state read and written once (the previous accept's
-    # positions replayed into the next buffer); 5 records written and the
-    # accepted ones read back; KV read over the context and 5 positions
-    # appended; 5 rows of logits
-    vbytes = (weights + 2 * (dn + conv) + 5 * rec + acc * rec + kvb * (ctx + 100) + 5 * kvb
-              + 5 * cfg.vocab * 4)
+    # the context grows by the accepted positions: its mean over the calls
+    vbytes = verify_bytes(cfg, ctx + kept / 2.0, 5, kept / calls)
     out["verify_5tok_ctx4096"] = {
         "calls_s": calls / (dev_ms / 1000.0), "ms_per_call": dev_ms / calls,
         "positions_s": 5 * calls / (dev_ms / 1000.0), "accepted_per_call": kept / calls,

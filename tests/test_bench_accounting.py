@@ -48,3 +48,20 @@ def test_prefill_flops_of_pp520():
     assert bench.matrix_params(cfg) == _layer_matrix_weights()
     flops = 2.0 * _layer_matrix_weights() * 520 + 2.0 * V * H
     assert flops == pytest.approx(504.744e9, rel=1e-5)
+
+
+def test_verify_bytes_of_one_call():
+    cfg = synth.hybrid_08b_config(max_ctx=4200)
+    bf16, f32 = 2, 4
+    ctx, n, replayed = 4096, 5, 1
+    weights = bench.decode_bytes(cfg, 0) - 2 * N_DN * NH * DV * DK * f32 \
+        - 2 * N_DN * CH * 3 * f32 - N_ATT * 2 * NKV * HD * bf16 - V * f32
+    state = 2 * (N_DN * NH * DV * DK * f32 + N_DN * CH * 3 * f32)  # read + replayed write
+    rec = N_DN * (NH * (DK + DV + 2) + CH) * f32                    # per position
+    kv = N_ATT * 2 * NKV * HD * bf16 * (ctx + n)                    # read ctx, append n
+    logits = n * V * f32
+    assert bench.weight_bytes(cfg) == weights
+    assert bench.verify_bytes(cfg, ctx, n, replayed) == \
+        weights + state + (n + replayed) * rec + kv + logits
+    # records are a few MB where 5 full state copies would be ~100 MB
+    assert (n + replayed) * rec < 5e6
